@@ -1,0 +1,441 @@
+#!/usr/bin/env python
+"""GPTQ layer-quantization throughput on B200.
+
+One step = the whole per-layer pass on one synthetic layer resident in HBM:
+  H = 2/N X^T X (tcgen05 SYRK) -> damping + U (Cholesky, triangular inverse)
+  -> the GPTQ column loop (lazy 128-column blocks + trailing updates)
+  -> packing of codes and zero points.
+Default workload: a Llama-7B attention projection, W 4096x4096 bf16 and X
+262,144 tokens x 4096 bf16 (the X stream alone is 2.15 GB, larger than L2),
+4-bit, group 128, damp 0.01, block 128.
+
+N GPUs (torchrun): every rank quantizes its own layer (a different seed); no
+collective on the data path (weak scaling); time = max over ranks.
+
+--impl reference times the fp64 CPU oracle (the only reference: the method's
+pages publish no code) on a bounded sample of the same workload.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GPTQ layer quant: weights/sec and ms per 4096×4096 layer; % of roofline"
+UNIT = "weights/s"
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="attn4096")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-tokens", type=int, default=8192, help="oracle sample: tokens for H")
+    ap.add_argument("--cpu-rows", type=int, default=32, help="oracle sample: rows through the column loop")
+    return ap.parse_args()
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK}, "measured"
+    except Exception:
+        return dict(FALLBACK), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id):
+        self.bus_id = (bus_id or "").lower()
+        self.proc = None
+        self.lines = []
+        self.t_start = self.t_stop = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                                          "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def mark(self, which):
+        setattr(self, "t_" + which, time.time())
+
+    def stop(self):
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        rows = []
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 10:
+                continue
+            if self.bus_id and not f[1].lower().endswith(self.bus_id[-12:]):
+                continue
+            try:
+                rows.append({"sm": float(f[2]), "max": float(f[3]), "power": float(f[4]),
+                             "hw_slowdown": f[6], "hw_thermal": f[7], "sw_thermal": f[8], "sw_power_cap": f[9]})
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        loaded = [r for r in rows if r["power"] > 300.0] or rows
+        reasons = set()
+        for r in loaded:
+            for k in ("hw_slowdown", "hw_thermal", "sw_thermal", "sw_power_cap"):
+                if r[k].lower() == "active":
+                    reasons.add({"hw_thermal": "hw_thermal_slowdown", "sw_thermal": "sw_thermal_slowdown"}.get(k, k))
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded), "sm_max_mhz": max(r["max"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(loaded)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle on a bounded sample
+# ---------------------------------------------------------------------------
+
+def oracle_sample(W_host, X_host, spec, tokens, rows):
+    """Times the fp64 oracle on a sample and scales each stage to the full layer.
+
+    H: `tokens` of the N tokens (cost grows with tokens) -> x N/tokens.
+    U: the full n x n factor (computed in full).
+    Column loop + packing: `rows` of the rows (rows are independent) -> x rows_total/rows.
+    """
+    import numpy as np
+
+    from oracle import gptq_oracle as go
+
+    n = spec.n
+    Xs = X_host[:tokens].double().numpy()
+    Ws = W_host[:rows].double().numpy()
+    t0 = time.perf_counter()
+    H = go.hessian(Xs, alpha=2.0 / tokens)
+    t1 = time.perf_counter()
+    prep = go.prepare(H, Ws, spec.damp, spec.act_order)
+    U = go.inverse_factor(prep["H"])
+    t2 = time.perf_counter()
+    res = go.gptq_quantize(prep["W"], U, spec.bits, spec.group, spec.block)
+    go.pack_codes(res["codes"], spec.bits)
+    t3 = time.perf_counter()
+    s_h = spec.n_tok / tokens
+    s_q = spec.rows / rows
+    full = (t1 - t0) * s_h + (t2 - t1) + (t3 - t2) * s_q
+    threads = None
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((i.get("num_threads") or 0) for i in threadpool_info()) or None
+    except Exception:
+        pass
+    cores = threads or len(os.sched_getaffinity(0))
+    sample = (f"fp64 oracle on {tokens} of {spec.n_tok} tokens for H (time x{s_h:g}), the full {n}x{n} factor, "
+              f"{rows} of {spec.rows} rows through the column loop and packing (time x{s_q:g}); "
+              f"measured {t3 - t0:.2f} s")
+    return {"value": spec.rows * n / full, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+            "est_s_per_layer": full, "stage_s": {"hessian_sample": t1 - t0, "factor": t2 - t1,
+                                                  "loop_and_pack_sample": t3 - t2}}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    with open(os.path.join(ROOT, "post_weight_quantization_accum_b200", "csrc", "hessian.cu"), "rb") as f:
+        h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload):
+    """Per-launch DRAM bytes of the SYRK kernel from an ncu capture, if it is
+    still the kernel that was captured (else None)."""
+    path = os.path.join(ROOT, "profiles", f"syrk_tc_kernel.{workload}.traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        if d.get("hessian_cu_sha256_16") == kernel_source_hash():
+            return float(d["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+def run_ours(args, world, rank, local):
+    import torch
+
+    import post_weight_quantization_accum_b200 as gq
+    import synth_inputs as si
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    base = si.SPECS[args.workload]
+    spec = si.scaled(base, seed=base.seed + 7919 * rank)
+    W, X = si.make_layer(spec, dev)
+    n, rows = spec.n, spec.rows
+    ng = gq.LIB.gptq_num_groups(n, spec.group)
+    alpha = 2.0 / spec.n_tok
+
+    H = torch.zeros((n, n), dtype=torch.float32, device=dev)
+    hdiag = torch.zeros(n, dtype=torch.float64, device=dev) if spec.act_order else None
+    U = torch.empty((n, n), dtype=torch.float32, device=dev)
+    perm = torch.empty(n, dtype=torch.int32, device=dev)
+    dead = torch.empty(n, dtype=torch.uint8, device=dev)
+    out = {"codes": torch.empty((rows, n), dtype=torch.uint8, device=dev),
+           "scales": torch.empty((rows, ng), dtype=torch.float32, device=dev),
+           "zeros": torch.empty((rows, ng), dtype=torch.uint8, device=dev),
+           "g_idx": torch.empty(n, dtype=torch.int32, device=dev)}
+    packed = torch.empty((rows, gq.LIB.gptq_packed_words_per_row(n, spec.bits)), dtype=torch.int32, device=dev)
+    packed_z = torch.empty((rows, gq.LIB.gptq_packed_words_per_row(ng, spec.bits)), dtype=torch.int32, device=dev)
+    ws_h = gq.workspace(gq.LIB.gptq_hessian_workspace_size(n, spec.n_tok), dev)
+    ws_p = gq.workspace(gq.LIB.gptq_prepare_workspace_size(n), dev)
+    ws_q = gq.workspace(gq.LIB.gptq_quantize_workspace_size(rows, n, spec.block), dev)
+
+    stream = torch.cuda.current_stream()
+    nev = 5
+
+    def step(evs):
+        H.zero_()
+        if hdiag is not None:
+            hdiag.zero_()
+        evs[0].record(stream)
+        gq.gptq_hessian_accum(H, X, alpha, hdiag=hdiag, ws=ws_h)
+        evs[1].record(stream)
+        gq.gptq_prepare_hinv(H, spec.damp, spec.act_order, hdiag=hdiag, perm=perm, dead=dead, U=U, ws=ws_p)
+        evs[2].record(stream)
+        gq.gptq_quantize_layer(W, U, spec.bits, spec.group, spec.block, perm=perm if spec.act_order else None,
+                               dead=dead, out=out, ws=ws_q)
+        evs[3].record(stream)
+        gq.gptq_pack(out["codes"], spec.bits, packed=packed)
+        gq.gptq_pack(out["zeros"], spec.bits, packed=packed_z)
+        evs[4].record(stream)
+
+    def new_events():
+        return [torch.cuda.Event(enable_timing=True) for _ in range(nev)]
+
+    for _ in range(args.warmup):
+        step(new_events())
+    torch.cuda.synchronize()
+    st = gq.gptq_get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {st}")
+
+    bus = None
+    try:
+        bus = torch.cuda.get_device_properties(dev).pci_bus_id
+    except Exception:
+        pass
+    sampler = ClockSampler(bus) if rank == 0 or world > 1 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    step_events = [new_events() for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = gq.gptq_kernel_launches()
+    t_start.record(stream)
+    for k in range(args.steps):
+        step(step_events[k])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    launches = gq.gptq_kernel_launches() - launches0
+    if sampler:
+        time.sleep(0.2)
+        sampler.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    stages = [[e[i].elapsed_time(e[i + 1]) for e in step_events] for i in range(nev - 1)]
+    stage_ms = [statistics.mean(s) for s in stages]
+    if dist is not None:
+        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    status = gq.gptq_get_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status after the timed region: {status}")
+
+    ms_per_step = elapsed_ms / args.steps
+    value = world * rows * n / (ms_per_step / 1e3)
+
+    pk, pk_src = peaks()
+    flops_syrk = float(n) * (n + 1) * spec.n_tok
+    achieved = flops_syrk / (stage_ms[0] / 1e3) / 1e12
+    traffic = measured_traffic(args.workload)
+    # algorithmic work of the factorization (for the per-stage table)
+    flops_factor = 2.0 * n ** 3 / 3.0
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{spec.name}: W {rows}x{n} {spec.w_dtype}, X {spec.n_tok} tokens x {n} bf16 "
+                               f"({spec.x_kind}), {spec.bits}-bit group {spec.group}, damp {spec.damp}, "
+                               f"block {spec.block}, act_order {spec.act_order}",
+                   "global_batch": spec.n_tok * world, "seq_len": 2048, "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2 (X alone is %.2f GB)" % (spec.n_tok * n * 2 / 1e9),
+                   "timing": "CUDA events on the launching stream; max over ranks"},
+        "roofline": {"bound": "tensor", "kernel": "syrk_tc_kernel (+ its finalize kernel)", "achieved": achieved,
+                     "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                     "frac": achieved / pk["bf16_tflops_sustained"], "traffic": traffic,
+                     "peak_source": f"{pk_src} bf16 sustained (kernel timed inside a long step)",
+                     "algorithmic_flops": flops_syrk},
+        "stages_ms": {"hessian": stage_ms[0], "prepare_hinv": stage_ms[1], "quantize_layer": stage_ms[2],
+                      "pack": stage_ms[3]},
+        "stage_rates": {"factor_tflops": flops_factor / (stage_ms[1] / 1e3) / 1e12,
+                        "column_loop_weights_per_s": rows * n / (stage_ms[2] / 1e3),
+                        "without_hessian_weights_per_s": rows * n / ((stage_ms[1] + stage_ms[2] + stage_ms[3]) / 1e3)},
+        "gpu_launches": launches,
+    }
+    if sampler:
+        result["clocks"] = sampler.summary()
+
+    if not args.no_e2e:
+        result["e2e"] = run_e2e(args, spec, W, X, dev, world, dist)
+
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = oracle_sample(W.cpu(), X[: args.cpu_tokens].cpu(), spec, args.cpu_tokens,
+                                               args.cpu_rows)
+        for k in ("est_s_per_layer", "stage_s"):
+            result["cpu_baseline"].pop(k, None)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result if rank == 0 else None
+
+
+def run_e2e(args, spec, W, X, dev, world, dist):
+    """The public call with host inputs: H2D of W and X, the layer pass, D2H of
+    the packed codes, packed zero points and scales, all inside the timing."""
+    import torch
+
+    import post_weight_quantization_accum_b200 as gq
+
+    Wh = W.cpu().pin_memory()
+    Xh = X.cpu().pin_memory()
+    stream = torch.cuda.current_stream()
+
+    def one():
+        Wd = Wh.to(dev, non_blocking=True)
+        Xd = Xh.to(dev, non_blocking=True)
+        out = gq.quantize_layer(Wd, Xd, bits=spec.bits, group=spec.group, damp=spec.damp, block=spec.block,
+                                act_order=spec.act_order)
+        res = (out["packed"].to("cpu", non_blocking=True), out["packed_zeros"].to("cpu", non_blocking=True),
+               out["scales"].to("cpu", non_blocking=True))
+        return res
+
+    res = one()
+    torch.cuda.synchronize()
+    h2d = Wh.numel() * Wh.element_size() + Xh.numel() * Xh.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in res)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(args.e2e_steps):
+        one()
+    e.record(stream)
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / args.e2e_steps
+    if dist is not None:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": world * spec.rows * spec.n / (ms / 1e3), "unit": UNIT, "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle
+# ---------------------------------------------------------------------------
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    import torch
+
+    import synth_inputs as si
+
+    spec = si.SPECS[args.workload]
+    # a bounded sample per step: 2048 tokens for H, 16 rows through the loop
+    tokens, rows = min(2048, spec.n_tok), min(16, spec.rows)
+    sub = si.scaled(spec, n_tok=tokens)
+    W = si.make_weights(spec, "cpu")[:rows]
+    X = si.make_activations(sub, "cpu")
+    for _ in range(args.warmup):
+        oracle_sample(W, X, spec, tokens, rows)
+    vals, ests, last = [], [], None
+    for _ in range(args.steps):
+        last = oracle_sample(W, X, spec, tokens, rows)
+        vals.append(last["value"])
+        ests.append(last["est_s_per_layer"])
+    value = statistics.mean(vals)
+    ms = statistics.mean(ests) * 1e3
+    cpu = {"value": value, "unit": UNIT, "cores": last["cores"], "kind": "oracle", "sample": last["sample"]}
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{spec.name} (oracle on a bounded sample, stages scaled to the full layer)",
+                       "global_batch": spec.n_tok, "seq_len": 2048, "parallelism": "cpu"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse_args()
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        res = run_reference(args, world, rank)
+    else:
+        res = run_ours(args, world, rank, local)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

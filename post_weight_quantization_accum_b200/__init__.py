@@ -1,0 +1,173 @@
+"""B200 (sm_100a) GPTQ per-layer quantization: Python binding of libgptq_b200.so.
+
+The functions below carry the names of the C entry points in include/gptq.h
+and only marshal arguments: torch supplies device memory and the current CUDA
+stream, the library's kernels do all of the work.  ``quantize_layer`` chains the
+four calls for one linear layer (the usual entry point for a user).
+"""
+import ctypes
+
+import torch
+
+from ._lib import GPTQ_BF16, GPTQ_F32, LIB, GptqError, check  # noqa: F401
+
+__all__ = [
+    "GptqError",
+    "gptq_hessian_accum",
+    "gptq_prepare_hinv",
+    "gptq_quantize_layer",
+    "gptq_quantize_rtn",
+    "gptq_pack",
+    "gptq_get_device_status",
+    "gptq_set_wait_limit_ns",
+    "gptq_kernel_launches",
+    "workspace",
+    "quantize_layer",
+]
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.float32:
+        return GPTQ_F32
+    if t.dtype == torch.bfloat16:
+        return GPTQ_BF16
+    raise TypeError(f"unsupported weight dtype {t.dtype}")
+
+
+def workspace(nbytes, device=None):
+    """A 256-byte aligned device buffer of at least ``nbytes`` (torch memory)."""
+    return torch.empty(max(int(nbytes), 1) + 256, dtype=torch.uint8, device=device or "cuda")
+
+
+def _ws_ptr(ws):
+    base = ws.data_ptr()
+    return ctypes.c_void_p((base + 255) & ~255), ws.numel() - ((-base) % 256)
+
+
+def gptq_get_device_status(stream=None):
+    return LIB.gptq_get_device_status(_stream(stream))
+
+
+def gptq_set_wait_limit_ns(ns):
+    LIB.gptq_set_wait_limit_ns(ctypes.c_uint64(ns))
+
+
+def gptq_kernel_launches():
+    return int(LIB.gptq_kernel_launches())
+
+
+def gptq_hessian_accum(H, X, alpha, hdiag=None, ws=None, stream=None):
+    """H += alpha * X^T X (X bf16 [n_tok, n] view with unit column stride); hdiag fp64 optional."""
+    if X.dtype != torch.bfloat16 or X.stride(1) != 1:
+        raise TypeError("X must be a bf16 matrix with contiguous rows")
+    n_tok, ldx = X.shape[0], X.stride(0)
+    n = H.shape[0]
+    need = LIB.gptq_hessian_workspace_size(n, n_tok)
+    if ws is None:
+        ws = workspace(need, H.device)
+    wp, wbytes = _ws_ptr(ws)
+    check("gptq_hessian_accum",
+          LIB.gptq_hessian_accum(_ptr(H), _ptr(hdiag), _ptr(X), n_tok, n, ldx, ctypes.c_float(alpha), wp,
+                                 wbytes, _stream(stream)))
+    return H
+
+
+def gptq_prepare_hinv(H, damp, act_order, hdiag=None, perm=None, dead=None, U=None, ws=None, stream=None):
+    """Returns (U, perm, dead) for the accumulated Hessian H (fp32 [n, n])."""
+    n = H.shape[0]
+    dev = H.device
+    U = U if U is not None else torch.empty((n, n), dtype=torch.float32, device=dev)
+    perm = perm if perm is not None else torch.empty(n, dtype=torch.int32, device=dev)
+    dead = dead if dead is not None else torch.empty(n, dtype=torch.uint8, device=dev)
+    if ws is None:
+        ws = workspace(LIB.gptq_prepare_workspace_size(n), dev)
+    wp, wbytes = _ws_ptr(ws)
+    check("gptq_prepare_hinv",
+          LIB.gptq_prepare_hinv(_ptr(H), _ptr(hdiag), n, ctypes.c_float(damp), int(bool(act_order)), _ptr(perm),
+                                _ptr(dead), _ptr(U), wp, wbytes, _stream(stream)))
+    return U, perm, dead
+
+
+def gptq_quantize_layer(W, U, bits, group, block=128, perm=None, dead=None, out=None, want_deq=False,
+                        want_loss=False, ws=None, stream=None):
+    """The GPTQ column loop; returns a dict of output tensors."""
+    rows, n = W.shape
+    dev = W.device
+    ng = LIB.gptq_num_groups(n, group)
+    out = dict(out or {})
+    out.setdefault("codes", torch.empty((rows, n), dtype=torch.uint8, device=dev))
+    out.setdefault("scales", torch.empty((rows, ng), dtype=torch.float32, device=dev))
+    out.setdefault("zeros", torch.empty((rows, ng), dtype=torch.uint8, device=dev))
+    out.setdefault("g_idx", torch.empty(n, dtype=torch.int32, device=dev))
+    if want_deq:
+        out.setdefault("deq", torch.empty((rows, n), dtype=torch.float32, device=dev))
+    if want_loss:
+        out.setdefault("row_loss", torch.empty(rows, dtype=torch.float32, device=dev))
+    if ws is None:
+        ws = workspace(LIB.gptq_quantize_workspace_size(rows, n, block), dev)
+    wp, wbytes = _ws_ptr(ws)
+    check("gptq_quantize_layer",
+          LIB.gptq_quantize_layer(_ptr(W), _dtype_code(W), rows, n, _ptr(U), _ptr(perm), _ptr(dead), bits, group,
+                                  block, _ptr(out["codes"]), _ptr(out["scales"]), _ptr(out["zeros"]),
+                                  _ptr(out.get("g_idx")), _ptr(out.get("deq")), _ptr(out.get("row_loss")), wp,
+                                  wbytes, _stream(stream)))
+    return out
+
+
+def gptq_quantize_rtn(W, bits, group, stream=None):
+    rows, n = W.shape
+    dev = W.device
+    ng = LIB.gptq_num_groups(n, group)
+    codes = torch.empty((rows, n), dtype=torch.uint8, device=dev)
+    scales = torch.empty((rows, ng), dtype=torch.float32, device=dev)
+    zeros = torch.empty((rows, ng), dtype=torch.uint8, device=dev)
+    check("gptq_quantize_rtn",
+          LIB.gptq_quantize_rtn(_ptr(W), _dtype_code(W), rows, n, bits, group, _ptr(codes), _ptr(scales),
+                                _ptr(zeros), _stream(stream)))
+    return {"codes": codes, "scales": scales, "zeros": zeros}
+
+
+def gptq_pack(codes, bits, packed=None, stream=None):
+    rows, n = codes.shape
+    words = LIB.gptq_packed_words_per_row(n, bits)
+    if packed is None:
+        packed = torch.empty((rows, words), dtype=torch.int32, device=codes.device)
+    check("gptq_pack", LIB.gptq_pack(_ptr(codes), rows, n, bits, _ptr(packed), _stream(stream)))
+    return packed
+
+
+def quantize_layer(W, X, bits=4, group=128, damp=0.01, block=128, act_order=False, want_deq=False,
+                   want_loss=False, stream=None):
+    """One linear layer end to end: H from X, U, the column loop, packing.
+
+    W: [rows, n] fp32/bf16 weights; X: [n_tok, n] bf16 calibration inputs.
+    Returns a dict with H, U, perm, codes, scales, zeros, g_idx, packed,
+    packed_zeros (and deq / row_loss when asked for).
+    """
+    n = W.shape[1]
+    dev = W.device
+    if X.stride(1) != 1 or X.stride(0) % 8 != 0 or X.data_ptr() % 16 != 0:
+        # the library streams X with TMA, whose row pitch must be a multiple
+        # of 16 bytes: hand it a row-padded copy
+        Xp = torch.zeros((X.shape[0], (n + 7) // 8 * 8), dtype=torch.bfloat16, device=dev)
+        Xp[:, :n] = X
+        X = Xp[:, :n]
+    H = torch.zeros((n, n), dtype=torch.float32, device=dev)
+    hdiag = torch.zeros(n, dtype=torch.float64, device=dev) if act_order else None
+    gptq_hessian_accum(H, X, 2.0 / X.shape[0], hdiag=hdiag, stream=stream)
+    U, perm, dead = gptq_prepare_hinv(H, damp, act_order, hdiag=hdiag, stream=stream)
+    out = gptq_quantize_layer(W, U, bits, group, block, perm=perm if act_order else None, dead=dead,
+                              want_deq=want_deq, want_loss=want_loss, stream=stream)
+    out["packed"] = gptq_pack(out["codes"], bits, stream=stream)
+    out["packed_zeros"] = gptq_pack(out["zeros"], bits, stream=stream)
+    out.update(H=H, U=U, perm=perm, dead=dead)
+    return out

@@ -1,0 +1,221 @@
+// C ABI of the library: argument validation, per-device state and dispatch to
+// the kernels in hessian.cu, hinv.cu, quantize.cu and pack.cu.  Nothing here
+// allocates device memory; every scratch byte comes from the caller.
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace gptq {
+
+size_t hessian_workspace_size(int n, int64_t n_tok);
+gptq_status hessian_accum(float* H, double* hdiag, const void* X, int64_t n_tok, int n, int64_t ldx, float alpha,
+                          void* ws, size_t ws_bytes, cudaStream_t stream);
+size_t prepare_workspace_size(int n);
+gptq_status prepare_hinv(const float* H, const double* hdiag, int n, float damp, int act_order, int32_t* perm,
+                         uint8_t* dead, float* U, void* ws, size_t ws_bytes, cudaStream_t st);
+size_t quantize_workspace_size(int64_t rows, int n);
+gptq_status quantize_layer(const void* W, gptq_dtype wdt, int64_t rows, int n, const float* U, const int32_t* perm,
+                           const uint8_t* dead, int bits, int group, int block, uint8_t* codes, float* scales,
+                           uint8_t* zeros, int32_t* g_idx, float* Wq_out, float* row_loss, void* ws, size_t ws_bytes,
+                           cudaStream_t st);
+gptq_status quantize_rtn(const void* W, gptq_dtype wdt, int64_t rows, int n, int bits, int group, uint8_t* codes,
+                         float* scales, uint8_t* zeros, cudaStream_t st);
+gptq_status pack_codes(const uint8_t* codes, int64_t rows, int n, int bits, uint32_t* packed, cudaStream_t st);
+
+// Status words of each device: [0] failures of asynchronous kernels (bounded
+// waits), [1] the factorization status of gptq_prepare_hinv.
+__device__ int g_status_words[2];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;
+
+std::mutex g_mutex;
+DeviceInfo g_info[kMaxDevices];
+bool g_have[kMaxDevices] = {};
+uint64_t g_wait_ns = kDefaultWaitNs;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+}  // namespace
+
+const DeviceInfo* device_info() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (!g_have[dev]) {
+    DeviceInfo d{};
+    d.device = dev;
+    if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return nullptr;
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_status_words) != cudaSuccess) return nullptr;
+    d.status = static_cast<int*>(addr);
+    if (cudaMemset(d.status, 0, sizeof(int) * 2) != cudaSuccess) return nullptr;
+    g_info[dev] = d;
+    g_have[dev] = true;
+  }
+  return &g_info[dev];
+}
+
+bool make_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
+                        uint64_t row_pitch_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_pitch_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  std::memset(map, 0, sizeof(*map));
+  return fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+uint64_t wait_limit_ns() { return g_wait_ns; }
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+}  // namespace gptq
+
+using namespace gptq;
+
+namespace {
+constexpr int kMaxN = 65535;
+bool valid_bits(int32_t b) { return b == 2 || b == 3 || b == 4 || b == 8; }
+bool valid_block(int32_t b) { return b >= 32 && b <= 128 && b % 32 == 0; }
+bool nests(int32_t group, int32_t block) { return group == 0 || block % group == 0 || group % block == 0; }
+}  // namespace
+
+extern "C" {
+
+const char* gptq_status_string(gptq_status s) {
+  switch (s) {
+    case GPTQ_OK: return "ok";
+    case GPTQ_ERR_INVALID_ARG: return "invalid argument";
+    case GPTQ_ERR_NOT_PD: return "damped Hessian is not positive definite";
+    case GPTQ_ERR_NONFINITE: return "non-finite value in the Hessian";
+    case GPTQ_ERR_CUDA: return "CUDA error";
+    case GPTQ_ERR_UNSUPPORTED: return "unsupported combination";
+    case GPTQ_ERR_TIMEOUT: return "bounded in-kernel wait ran out";
+  }
+  return "unknown status";
+}
+
+int32_t gptq_version(void) { return 100; }
+
+uint64_t gptq_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+void gptq_set_wait_limit_ns(uint64_t ns) { g_wait_ns = ns == UINT64_MAX ? 2000000000ull : ns; }
+
+gptq_status gptq_get_device_status(void* stream) {
+  const DeviceInfo* info = device_info();
+  if (info == nullptr) return GPTQ_ERR_CUDA;
+  int v = 0;
+  cudaStream_t st = as_stream(stream);
+  if (cudaMemcpyAsync(&v, info->status, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return GPTQ_ERR_CUDA;
+  if (cudaMemsetAsync(info->status, 0, sizeof(int), st) != cudaSuccess) return GPTQ_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return GPTQ_ERR_CUDA;
+  return static_cast<gptq_status>(v);
+}
+
+size_t gptq_hessian_workspace_size(int32_t n, int64_t n_tok) {
+  if (n < 1 || n > kMaxN || n_tok < 0) return 0;
+  return hessian_workspace_size(n, n_tok);
+}
+
+gptq_status gptq_hessian_accum(float* H, double* hdiag, const void* X, int64_t n_tok, int32_t n, int64_t ldx,
+                               float alpha, void* ws, size_t ws_bytes, void* stream) {
+  if (H == nullptr || n < 1 || n > kMaxN || n_tok < 0 || n_tok > (int64_t(1) << 31) - 128 || !std::isfinite(alpha))
+    return GPTQ_ERR_INVALID_ARG;
+  if (n_tok == 0) return GPTQ_OK;
+  if (X == nullptr || ldx < n || ldx % 8 != 0 || !aligned(X, 16) || !aligned(H, 16)) return GPTQ_ERR_INVALID_ARG;
+  if (ws == nullptr || !aligned(ws, 256) || ws_bytes < hessian_workspace_size(n, n_tok)) return GPTQ_ERR_INVALID_ARG;
+  if (hdiag != nullptr && !aligned(hdiag, 8)) return GPTQ_ERR_INVALID_ARG;
+  return hessian_accum(H, hdiag, X, n_tok, n, ldx, alpha, ws, ws_bytes, as_stream(stream));
+}
+
+size_t gptq_prepare_workspace_size(int32_t n) {
+  if (n < 1 || n > kMaxN) return 0;
+  return prepare_workspace_size(n);
+}
+
+gptq_status gptq_prepare_hinv(const float* H, const double* hdiag, int32_t n, float damp, int32_t act_order,
+                              int32_t* perm, uint8_t* dead, float* U, void* ws, size_t ws_bytes, void* stream) {
+  if (H == nullptr || U == nullptr || n < 1 || n > kMaxN || !std::isfinite(damp) || damp < 0.0f)
+    return GPTQ_ERR_INVALID_ARG;
+  if (act_order && perm == nullptr) return GPTQ_ERR_INVALID_ARG;
+  if (ws == nullptr || !aligned(ws, 256) || ws_bytes < prepare_workspace_size(n)) return GPTQ_ERR_INVALID_ARG;
+  return prepare_hinv(H, hdiag, n, damp, act_order ? 1 : 0, perm, dead, U, ws, ws_bytes, as_stream(stream));
+}
+
+size_t gptq_quantize_workspace_size(int64_t rows, int32_t n, int32_t block) {
+  if (rows < 0 || n < 1 || n > kMaxN || !valid_block(block)) return 0;
+  return quantize_workspace_size(rows, n);
+}
+
+int32_t gptq_num_groups(int32_t n, int32_t group) {
+  if (n < 1 || group < 0) return 0;
+  return group == 0 ? 1 : static_cast<int32_t>((n + group - 1) / group);
+}
+
+gptq_status gptq_quantize_layer(const void* W, gptq_dtype wdt, int64_t rows, int32_t n, const float* U,
+                                const int32_t* perm, const uint8_t* dead, int32_t bits, int32_t group, int32_t block,
+                                uint8_t* codes, float* scales, uint8_t* zeros, int32_t* g_idx, float* Wq_out,
+                                float* row_loss, void* ws, size_t ws_bytes, void* stream) {
+  if (rows < 0 || n < 1 || n > kMaxN || !valid_bits(bits) || !valid_block(block) || group < 0 || group > n)
+    return GPTQ_ERR_INVALID_ARG;
+  if (wdt != GPTQ_F32 && wdt != GPTQ_BF16) return GPTQ_ERR_INVALID_ARG;
+  if (!nests(group, block)) return GPTQ_ERR_UNSUPPORTED;
+  if (rows == 0) return GPTQ_OK;
+  if (W == nullptr || U == nullptr || codes == nullptr || scales == nullptr || zeros == nullptr)
+    return GPTQ_ERR_INVALID_ARG;
+  if (ws == nullptr || !aligned(ws, 256) || ws_bytes < quantize_workspace_size(rows, n)) return GPTQ_ERR_INVALID_ARG;
+  return quantize_layer(W, wdt, rows, n, U, perm, dead, bits, group, block, codes, scales, zeros, g_idx, Wq_out,
+                        row_loss, ws, ws_bytes, as_stream(stream));
+}
+
+gptq_status gptq_quantize_rtn(const void* W, gptq_dtype wdt, int64_t rows, int32_t n, int32_t bits, int32_t group,
+                              uint8_t* codes, float* scales, uint8_t* zeros, void* stream) {
+  if (rows < 0 || n < 1 || n > kMaxN || !valid_bits(bits) || group < 0 || group > n) return GPTQ_ERR_INVALID_ARG;
+  if (wdt != GPTQ_F32 && wdt != GPTQ_BF16) return GPTQ_ERR_INVALID_ARG;
+  if (rows == 0) return GPTQ_OK;
+  if (W == nullptr || codes == nullptr || scales == nullptr || zeros == nullptr) return GPTQ_ERR_INVALID_ARG;
+  return quantize_rtn(W, wdt, rows, n, bits, group, codes, scales, zeros, as_stream(stream));
+}
+
+int32_t gptq_packed_words_per_row(int32_t n, int32_t bits) {
+  if (n < 0 || !valid_bits(bits)) return 0;
+  return bits * ((n + 31) / 32);
+}
+
+gptq_status gptq_pack(const uint8_t* codes, int64_t rows, int32_t n, int32_t bits, uint32_t* packed, void* stream) {
+  if (rows < 0 || n < 1 || !valid_bits(bits)) return GPTQ_ERR_INVALID_ARG;
+  if (rows == 0) return GPTQ_OK;
+  if (codes == nullptr || packed == nullptr || !aligned(packed, 4)) return GPTQ_ERR_INVALID_ARG;
+  return pack_codes(codes, rows, n, bits, packed, as_stream(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,76 @@
+"""The C-ABI library loads on the CPU and exports every entry point its header
+declares; pure (non-compute) calls answer without a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gptq.h")
+LIB = os.path.join(ROOT, "post_weight_quantization_accum_b200", "libgptq_b200.so")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gptq_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(LIB):
+        from post_weight_quantization_accum_b200 import build as b
+        b.build()
+    return ctypes.CDLL(LIB)
+
+
+def test_header_declares_the_four_calls():
+    names = declared_functions()
+    for n in ("gptq_hessian_accum", "gptq_prepare_hinv", "gptq_quantize_layer", "gptq_pack"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_pure_calls(lib):
+    lib.gptq_packed_words_per_row.restype = ctypes.c_int32
+    assert lib.gptq_packed_words_per_row(4096, 4) == 512
+    assert lib.gptq_packed_words_per_row(33, 3) == 6
+    assert lib.gptq_packed_words_per_row(10, 5) == 0
+    assert lib.gptq_num_groups(4096, 128) == 32
+    assert lib.gptq_num_groups(100, 0) == 1
+    assert lib.gptq_num_groups(129, 64) == 3
+    lib.gptq_status_string.restype = ctypes.c_char_p
+    assert lib.gptq_status_string(2) == b"damped Hessian is not positive definite"
+    assert lib.gptq_version() == 100
+
+
+def test_invalid_arguments_rejected_before_any_launch(lib):
+    P = ctypes.c_void_p
+    f = lib.gptq_quantize_layer
+    f.argtypes = [P, ctypes.c_int, ctypes.c_int64, ctypes.c_int32, P, P, P, ctypes.c_int32, ctypes.c_int32,
+                  ctypes.c_int32, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+    fake = P(256)
+    # bits 5, block 48, group/block not nesting, bad dtype
+    assert f(fake, 0, 8, 64, fake, None, None, 5, 0, 128, fake, fake, fake, None, None, None, fake, 1 << 30, None) == 1
+    assert f(fake, 0, 8, 64, fake, None, None, 4, 0, 48, fake, fake, fake, None, None, None, fake, 1 << 30, None) == 1
+    assert f(fake, 0, 8, 96, fake, None, None, 4, 48, 64, fake, fake, fake, None, None, None, fake, 1 << 30, None) == 5
+    assert f(fake, 7, 8, 64, fake, None, None, 4, 0, 64, fake, fake, fake, None, None, None, fake, 1 << 30, None) == 1
+    g = lib.gptq_pack
+    g.argtypes = [P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, P, P]
+    assert g(None, 4, 64, 4, fake, None) == 1
+    assert g(fake, 4, 64, 6, fake, None) == 1
+    h = lib.gptq_hessian_accum
+    h.argtypes = [P, P, P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, P, ctypes.c_size_t, P]
+    assert h(fake, None, fake, 128, 64, 60, 1.0, fake, 1 << 30, None) == 1    # ldx < n
+    assert h(fake, None, fake, 128, 64, 68, 1.0, fake, 1 << 30, None) == 1    # ldx % 8
+    assert h(fake, None, P(258), 128, 64, 64, 1.0, fake, 1 << 30, None) == 1  # X alignment
+    assert h(fake, None, fake, 0, 64, 64, 1.0, None, 0, None) == 0            # no tokens: no-op
+    p = lib.gptq_prepare_hinv
+    p.argtypes = [P, P, ctypes.c_int32, ctypes.c_float, ctypes.c_int32, P, P, P, P, ctypes.c_size_t, P]
+    assert p(fake, None, 64, -0.1, 0, None, None, fake, fake, 1 << 30, None) == 1
+    assert p(fake, None, 64, 0.01, 1, None, None, fake, fake, 1 << 30, None) == 1  # act-order needs perm

@@ -1,0 +1,256 @@
+"""CUDA path vs the fp64 oracle, element by element, on seeded inputs.
+
+Bars (from the benchmark spec of the method's tolerances):
+  * H: relative Frobenius error <= 1e-3 against the oracle's fp64 H of the
+    same bf16-rounded X (expected ~1e-6: products are exact, fp32 sums).
+  * whole layer: >= 99.9% identical integer codes and ||(W-Q)X||_F^2 within
+    1e-3 relative of the oracle's.
+  * the grid applied to an identical column is bit-exact (RTN, and the column
+    loop with U = I) against the oracle's float32 grid.
+  * packing and permutation work are integer work: bit-exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import gptq_oracle as go
+import synth_inputs as si
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import post_weight_quantization_accum_b200 as gq
+
+
+def np64(t):
+    return t.detach().cpu().to(torch.float64).numpy()
+
+
+def npx(t):
+    return t.detach().cpu().numpy()
+
+
+def rel_fro(a, b):
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+# ---------------------------------------------------------------------------
+# round-to-nearest and the grid: bit-exact
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+@pytest.mark.parametrize("group", [0, 32, 128, 100])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_rtn_bit_exact(bits, group, dtype):
+    g = torch.Generator(device="cuda").manual_seed(bits * 100 + group)
+    W = (torch.randn((37, 300), generator=g, device="cuda") * 0.02).to(dtype)
+    W[3, :] = 0.0                      # an all-zero row
+    W[5, :64] = torch.abs(W[5, :64])   # groups without negative values
+    out = gq.gptq_quantize_rtn(W, bits, group)
+    ref = go.rtn_quantize_f32(npx(W.float()), bits, group)
+    assert np.array_equal(npx(out["codes"]).astype(np.int64), ref["codes"])
+    assert np.array_equal(npx(out["scales"]), ref["scales"].astype(np.float32))
+    assert np.array_equal(npx(out["zeros"]).astype(np.float32), ref["zeros"])
+
+
+@pytest.mark.parametrize("bits,group,block", [(4, 128, 128), (3, 64, 128), (2, 32, 64), (8, 0, 32), (4, 256, 128)])
+def test_column_loop_with_identity_factor_is_rtn(bits, group, block):
+    g = torch.Generator(device="cuda").manual_seed(7)
+    n = 512
+    W = torch.randn((50, n), generator=g, device="cuda") * 0.02
+    U = torch.eye(n, device="cuda")
+    out = gq.gptq_quantize_layer(W, U, bits, group, block, want_deq=True, want_loss=True)
+    ref = go.rtn_quantize_f32(npx(W), bits, group)
+    assert np.array_equal(npx(out["codes"]).astype(np.int64), ref["codes"])
+    assert np.array_equal(npx(out["scales"]), ref["scales"].astype(np.float32))
+    assert np.array_equal(npx(out["deq"]), ref["deq"])
+
+
+# ---------------------------------------------------------------------------
+# packing: bit-exact
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+@pytest.mark.parametrize("n", [1, 31, 32, 33, 96, 4096])
+def test_pack_bit_exact(bits, n):
+    g = torch.Generator(device="cuda").manual_seed(bits + n)
+    codes = torch.randint(0, 1 << bits, (9, n), generator=g, device="cuda", dtype=torch.int32).to(torch.uint8)
+    packed = gq.gptq_pack(codes, bits)
+    ref = go.pack_codes(npx(codes).astype(np.int64), bits)
+    assert np.array_equal(npx(packed).view(np.uint32), ref)
+
+
+# ---------------------------------------------------------------------------
+# Hessian accumulation
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("n,ldx,n_tok", [(64, 64, 1), (128, 128, 63), (256, 256, 2048), (320, 320, 1000),
+                                         (127, 128, 65), (1000, 1000, 3000), (129, 136, 4097)])
+def test_hessian_matches_fp64(n, ldx, n_tok):
+    g = torch.Generator(device="cuda").manual_seed(n * 7 + n_tok)
+    Xfull = torch.randn((n_tok, ldx), generator=g, device="cuda").to(torch.bfloat16)
+    X = Xfull[:, :n]
+    scales = torch.exp(torch.randn(n, generator=g, device="cuda"))
+    Xfull[:, :n] = (X.float() * scales).to(torch.bfloat16)
+    H = torch.zeros((n, n), device="cuda")
+    hdiag = torch.zeros(n, dtype=torch.float64, device="cuda")
+    alpha = 2.0 / n_tok
+    gq.gptq_hessian_accum(H, Xfull[:, :n], alpha, hdiag=hdiag)
+    torch.cuda.synchronize()
+    Xh = np64(Xfull[:, :n])
+    ref = go.hessian(Xh, alpha=np.float32(alpha))
+    Hg = np64(H)
+    assert rel_fro(Hg, ref) <= 1e-3
+    assert rel_fro(Hg, ref) <= 1e-5  # what fp32 accumulation of exact products gives
+    assert np.array_equal(Hg, Hg.T)
+    np.testing.assert_allclose(np64(hdiag), np.diag(ref), rtol=1e-12)
+    # deterministic and accumulating
+    H2 = torch.zeros_like(H)
+    gq.gptq_hessian_accum(H2, Xfull[:, :n], alpha)
+    assert torch.equal(H, H2)
+    gq.gptq_hessian_accum(H2, Xfull[:, :n], alpha)
+    assert rel_fro(np64(H2), 2 * ref) <= 1e-5
+
+
+def test_hessian_chunked_equals_oneshot():
+    spec = si.scaled(si.SPECS["attn4096"], rows=8, n=384, n_tok=6000)
+    X = si.make_activations(spec, "cuda")
+    H1 = torch.zeros((384, 384), device="cuda")
+    gq.gptq_hessian_accum(H1, X, 2.0 / 6000)
+    H2 = torch.zeros((384, 384), device="cuda")
+    for a in range(0, 6000, 1024):
+        gq.gptq_hessian_accum(H2, X[a:a + 1024], 2.0 / 6000)
+    assert rel_fro(np64(H2), np64(H1)) <= 1e-6
+
+
+# ---------------------------------------------------------------------------
+# damping, act-order and U
+# ---------------------------------------------------------------------------
+
+def _spd_from_x(n, n_tok, seed, dead=()):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    X = (torch.randn((n_tok, n), generator=g, device="cuda") * torch.exp(torch.randn(n, generator=g, device="cuda")))
+    X[:, list(dead)] = 0.0
+    X = X.to(torch.bfloat16)
+    Hx = go.hessian(np64(X))
+    return X, Hx
+
+
+@pytest.mark.parametrize("n,act_order", [(64, False), (200, True), (256, False), (515, True), (1024, False)])
+def test_prepare_matches_oracle(n, act_order):
+    X, Hx = _spd_from_x(n, 4 * n, seed=n, dead=(3,))
+    H32 = torch.tensor(Hx.astype(np.float32), device="cuda")
+    U, perm, dead = gq.gptq_prepare_hinv(H32, 0.01, act_order)
+    torch.cuda.synchronize()
+    prep = go.prepare(Hx.astype(np.float32).astype(np.float64), np.zeros((1, n)), 0.01, act_order)
+    assert np.array_equal(npx(perm).astype(np.int64), prep["perm"])
+    assert npx(dead).tolist() == prep["dead"].astype(np.uint8).tolist()
+    Uref = go.inverse_factor(prep["H"])
+    Ug = np64(U)
+    assert np.all(np.tril(Ug, -1) == 0.0)
+    assert rel_fro(Ug, Uref) <= 1e-4
+    # U^T U H' = I on random probes
+    rng = np.random.default_rng(n)
+    for _ in range(3):
+        v = rng.standard_normal(n)
+        r = Ug.T @ (Ug @ (prep["H"] @ v)) - v
+        assert np.linalg.norm(r) / np.linalg.norm(v) <= 1e-3
+
+
+def test_prepare_not_positive_definite():
+    n = 96
+    g = torch.Generator(device="cuda").manual_seed(1)
+    X = torch.randn((40, n), generator=g, device="cuda").to(torch.bfloat16)   # rank 40 < 96
+    H = torch.zeros((n, n), device="cuda")
+    gq.gptq_hessian_accum(H, X, 2.0 / 40)
+    with pytest.raises(gq.GptqError) as ei:
+        gq.gptq_prepare_hinv(H, 0.0, False)
+    assert ei.value.status == "GPTQ_ERR_NOT_PD"
+    H[5, 7] = float("nan")
+    H[7, 5] = float("nan")
+    with pytest.raises(gq.GptqError) as ei:
+        gq.gptq_prepare_hinv(H, 0.01, False)
+    assert ei.value.status == "GPTQ_ERR_NONFINITE"
+
+
+# ---------------------------------------------------------------------------
+# whole layer against the oracle
+# ---------------------------------------------------------------------------
+
+def _layer_parity(spec, dead=()):
+    W, X = si.make_layer(spec, "cuda")
+    if dead:
+        X[:, list(dead)] = 0
+    out = gq.quantize_layer(W, X, bits=spec.bits, group=spec.group, damp=spec.damp, block=spec.block,
+                            act_order=spec.act_order, want_deq=True, want_loss=True)
+    torch.cuda.synchronize()
+    Xh = np64(X)
+    Wh = np64(W)
+    ref = go.gptq_layer(Wh, X=Xh, bits=spec.bits, group=spec.group, damp=spec.damp, block=spec.block,
+                        act_order=spec.act_order)
+    codes = npx(out["codes"]).astype(np.int64)
+    agree = float(np.mean(codes == ref["codes"]))
+    S = Xh.T @ Xh
+    err_gpu = go.layer_output_error(Wh, np64(out["deq"]), S)
+    err_ref = go.layer_output_error(Wh, ref["deq"], S)
+    return out, ref, agree, err_gpu, err_ref
+
+
+@pytest.mark.parametrize("name,rows,n,n_tok", [
+    ("layer256", 256, 256, 2048),          # the 256x256 fp32 configuration in full
+    ("attn4096", 96, 384, 4096),           # attention-projection structure, several blocks + groups
+    ("mlp_up", 64, 320, 3000),             # 3-bit g128 act-order, ragged last block
+    ("mlp_down", 48, 448, 3000),           # half-normal inputs with zeros, act-order
+    ("fc2_g64_2b", 40, 256, 2000),         # 2-bit g64
+])
+def test_layer_matches_oracle(name, rows, n, n_tok):
+    spec = si.scaled(si.SPECS[name], rows=rows, n=n, n_tok=n_tok)
+    out, ref, agree, err_gpu, err_ref = _layer_parity(spec)
+    assert agree >= 0.999, agree
+    assert abs(err_gpu - err_ref) <= 1e-3 * err_ref, (err_gpu, err_ref)
+    if spec.act_order:
+        assert np.array_equal(npx(out["perm"]).astype(np.int64), ref["perm"])
+        assert np.array_equal(npx(out["g_idx"]).astype(np.int64), ref["g_idx"])
+    # scales: same group structure, values within fp32-vs-fp64 drift
+    sg, sr = npx(out["scales"]), ref["scales"]
+    assert np.mean(np.isclose(sg, sr, rtol=1e-4)) >= 0.999
+    # loss identity on the GPU's own outputs: sum e^2 vs (w-q)^T H' (w-q)
+    np.testing.assert_allclose(npx(out["row_loss"]), ref["row_loss"], rtol=2e-2)
+
+
+@pytest.mark.parametrize("block", [32, 64, 128])
+@pytest.mark.parametrize("group", [0, 32, 128])
+def test_block_size_invariance_on_gpu(block, group):
+    if group and not (block % group == 0 or group % block == 0):
+        pytest.skip("group and block must nest")
+    spec = si.scaled(si.SPECS["attn4096"], rows=64, n=256, n_tok=2048, block=block, group=group)
+    out, ref, agree, err_gpu, err_ref = _layer_parity(spec)
+    assert agree >= 0.999
+    assert abs(err_gpu - err_ref) <= 1e-3 * err_ref
+
+
+def test_dead_columns_and_bf16_weights():
+    spec = si.scaled(si.SPECS["attn4096"], rows=32, n=192, n_tok=1500, group=64)
+    out, ref, agree, err_gpu, err_ref = _layer_parity(spec, dead=(0, 77, 191))
+    assert agree >= 0.999
+    assert npx(out["dead"])[[0, 77, 191]].tolist() == [1, 1, 1]
+    assert np.all(npx(out["deq"])[:, [0, 77, 191]] == 0.0)
+
+
+def test_tiny_and_ragged_shapes():
+    for rows, n in [(1, 1), (1, 31), (3, 33), (5, 129), (2, 200)]:
+        spec = si.scaled(si.SPECS["layer256"], rows=rows, n=n, n_tok=300)
+        out, ref, agree, err_gpu, err_ref = _layer_parity(spec)
+        assert agree >= 0.99 or np.sum(npx(out["codes"]) != ref["codes"]) <= 1, (rows, n)
+        assert abs(err_gpu - err_ref) <= 1e-3 * max(err_ref, 1e-30) + 1e-12
+
+
+def test_packed_outputs_roundtrip():
+    spec = si.scaled(si.SPECS["attn4096"], rows=16, n=256, n_tok=1024, bits=3)
+    W, X = si.make_layer(spec, "cuda")
+    out = gq.quantize_layer(W, X, bits=3, group=128)
+    torch.cuda.synchronize()
+    codes = npx(out["codes"]).astype(np.int64)
+    assert np.array_equal(go.unpack_codes(npx(out["packed"]).view(np.uint32), 256, 3), codes)
+    assert np.array_equal(go.unpack_codes(npx(out["packed_zeros"]).view(np.uint32), 2, 3),
+                          npx(out["zeros"]).astype(np.int64))
