@@ -39,6 +39,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="attn4096")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the calibration token count (small profiling captures only)")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -69,15 +71,16 @@ def peaks():
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
-    QUERY = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi samples (every 100 ms) of the GPU a process runs on."""
+
+    QUERY = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, bus_id):
-        self.bus_id = (bus_id or "").lower()
+    def __init__(self, uuid):
+        self.uuid = (uuid or "").lower()
         self.proc = None
         self.lines = []
-        self.t_start = self.t_stop = None
 
     def start(self):
         try:
@@ -85,9 +88,6 @@ class ClockSampler:
                                           "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
-
-    def mark(self, which):
-        setattr(self, "t_" + which, time.time())
 
     def stop(self):
         if self.proc is None:
@@ -106,7 +106,7 @@ class ClockSampler:
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 10:
                 continue
-            if self.bus_id and not f[1].lower().endswith(self.bus_id[-12:]):
+            if self.uuid and self.uuid not in f[1].lower():
                 continue
             try:
                 rows.append({"sm": float(f[2]), "max": float(f[3]), "power": float(f[4]),
@@ -117,10 +117,11 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
         loaded = [r for r in rows if r["power"] > 300.0] or rows
         reasons = set()
+        names = {"hw_thermal": "hw_thermal_slowdown", "sw_thermal": "sw_thermal_slowdown"}
         for r in loaded:
             for k in ("hw_slowdown", "hw_thermal", "sw_thermal", "sw_power_cap"):
                 if r[k].lower() == "active":
-                    reasons.add({"hw_thermal": "hw_thermal_slowdown", "sw_thermal": "sw_thermal_slowdown"}.get(k, k))
+                    reasons.add(names.get(k, k))
         return {"sm_mhz": statistics.median(r["sm"] for r in loaded), "sm_max_mhz": max(r["max"] for r in rows),
                 "reasons": sorted(reasons), "samples": len(loaded)}
 
@@ -211,7 +212,7 @@ def run_ours(args, world, rank, local):
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
     base = si.SPECS[args.workload]
-    spec = si.scaled(base, seed=base.seed + 7919 * rank)
+    spec = si.scaled(base, seed=base.seed + 7919 * rank, n_tok=args.tokens or base.n_tok)
     W, X = si.make_layer(spec, dev)
     n, rows = spec.n, spec.rows
     ng = gq.LIB.gptq_num_groups(n, spec.group)
@@ -261,12 +262,12 @@ def run_ours(args, world, rank, local):
     if st != 0:
         raise RuntimeError(f"device status after warm-up: {st}")
 
-    bus = None
+    uuid = None
     try:
-        bus = torch.cuda.get_device_properties(dev).pci_bus_id
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
     except Exception:
         pass
-    sampler = ClockSampler(bus) if rank == 0 or world > 1 else None
+    sampler = ClockSampler(uuid)
     if sampler:
         sampler.start()
         time.sleep(0.3)

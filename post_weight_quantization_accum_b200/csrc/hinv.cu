@@ -424,7 +424,7 @@ gptq_status prepare_hinv(const float* H, const double* hdiag, int n, float damp,
     launch(tri_gemm_left_lower_kernel, g, 256, 0, st, U, T, n, s);
   }
   const int64_t nn = static_cast<int64_t>(n) * n;
-  launch(rotate180_kernel, static_cast<unsigned>(ceil_div(nn / 2, 256)), 256, 0, st, U, nn);
+  if (nn >= 2) launch(rotate180_kernel, static_cast<unsigned>(ceil_div(nn / 2, 256)), 256, 0, st, U, nn);
   if (launch_status() != GPTQ_OK) return GPTQ_ERR_CUDA;
 
   int fs = 0;

@@ -105,7 +105,14 @@ __global__ void __launch_bounds__(kRowsPerCta * 32) gptq_block_kernel(BlockArgs 
     ek[m] = 0.0f;
     qk[m] = 0.0f;
   }
+  // A group that began in an earlier block keeps the (scale, zero) that
+  // block fixed; they are read back from the outputs.
   GridParams gp{1.0f, 0.0f};
+  if (a.i1 % a.G != 0) {
+    const int g = a.i1 / a.G;
+    gp.scale = a.scales[r * a.n_groups + g];
+    gp.zero = static_cast<float>(a.zeros[r * a.n_groups + g]);
+  }
   float loss = 0.0f;
 
 #pragma unroll
