@@ -214,6 +214,33 @@ gptq_status gptq_quantize_layer(const void* W, gptq_dtype wdt, int64_t rows,
                                 float* row_loss, void* ws, size_t ws_bytes,
                                 void* stream);
 
+/* Allocation-free variant of gptq_quantize_layer.
+ *
+ * The pages have no counterpart to this call; it exists for callers that
+ * cannot provide a workspace: code that must not call cudaMalloc or cudaFree
+ * (cudaFree synchronizes the whole device), plugins inside a host application
+ * that owns all device memory through its own pool, and callers not allowed
+ * to allocate at all.  Same arguments, outputs and kernels as
+ * gptq_quantize_layer, minus ws / ws_bytes: the scratch is a fixed device array
+ * of GPTQ_NOALLOC_SCRATCH_BYTES compiled into the library, which every GPU that
+ * loads the library holds until the process exits.
+ *   - Layers whose gptq_quantize_workspace_size(rows, n, block) exceeds
+ *     GPTQ_NOALLOC_SCRATCH_BYTES are rejected with GPTQ_ERR_INVALID_ARG
+ *     (e.g. 1024 x 2048 fits, 2048 x 2048 does not).
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls share the array: calls whose kernels overlap on the GPU race
+ *     and give wrong results.  The array keeps the last call's contents; the
+ *     column loop writes every scratch byte before reading it.
+ *   - It allocates nothing (no cudaMalloc, cudaFree or allocating routine). */
+#define GPTQ_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+gptq_status gptq_quantize_layer_noalloc(const void* W, gptq_dtype wdt, int64_t rows,
+                                        int32_t n, const float* U, const int32_t* perm,
+                                        const uint8_t* dead, int32_t bits, int32_t group,
+                                        int32_t block, uint8_t* codes, float* scales,
+                                        uint8_t* zeros, int32_t* g_idx, float* Wq_out,
+                                        float* row_loss, void* stream);
+
 /* Round-to-nearest on the same grid (groups of `group` original columns, 0 =
  * per row); the baseline GPTQ improves on (knowledge note, "Why It Exists").
  * Outputs as in gptq_quantize_layer.  Needs no workspace. */
