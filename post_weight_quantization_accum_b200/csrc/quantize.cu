@@ -79,14 +79,34 @@ struct BlockArgs {
   float* row_loss;       // [rows] or nullptr
 };
 
-__global__ void __launch_bounds__(kRowsPerCta * 32) gptq_block_kernel(BlockArgs a) {
+__global__ void __launch_bounds__(kRowsPerCta * 32, 1) gptq_block_kernel(BlockArgs a) {
   extern __shared__ float dyn_smem[];
   float* us = dyn_smem;              // [kBMax][kBMax] U tile of the block
   float* rdiag = dyn_smem + kBMax * kBMax;
   const int bw = a.bw;
-  for (int e = threadIdx.x; e < bw * bw; e += blockDim.x) {
-    const int j = e / bw, k = e % bw;
-    us[j * kBMax + k] = a.U[static_cast<size_t>(a.i1 + j) * a.n + a.i1 + k];
+  // U tile: each thread issues a batch of loads before storing any of them,
+  // 16-byte loads when the rows allow it.
+  if (bw == kBMax && a.n % 4 == 0) {
+    constexpr int kVec = kBMax * kBMax / 4 / (kRowsPerCta * 32);  // 8 float4 per thread
+    float4 v[kVec];
+#pragma unroll
+    for (int q = 0; q < kVec; ++q) {
+      const int e = threadIdx.x + q * kRowsPerCta * 32, j = e / (kBMax / 4), k4 = e % (kBMax / 4);
+      v[q] = __ldg(reinterpret_cast<const float4*>(a.U + static_cast<size_t>(a.i1 + j) * a.n + a.i1) + k4);
+    }
+#pragma unroll
+    for (int q = 0; q < kVec; ++q) reinterpret_cast<float4*>(us)[threadIdx.x + q * kRowsPerCta * 32] = v[q];
+  } else {
+    for (int e0 = 0; e0 < kBMax * kBMax; e0 += 8 * kRowsPerCta * 32) {
+      float v[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int e = e0 + threadIdx.x + q * kRowsPerCta * 32, j = e / kBMax, k = e % kBMax;
+        v[q] = (j < bw && k < bw) ? __ldg(a.U + static_cast<size_t>(a.i1 + j) * a.n + a.i1 + k) : 0.0f;
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) us[e0 + threadIdx.x + q * kRowsPerCta * 32] = v[q];
+    }
   }
   __syncthreads();
   for (int j = threadIdx.x; j < bw; j += blockDim.x) rdiag[j] = 1.0f / us[j * kBMax + j];
@@ -188,13 +208,21 @@ __global__ void __launch_bounds__(256) trailing_update_kernel(float* __restrict_
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
   float acc[8][8] = {};
   for (int k0 = 0; k0 < bw; k0 += TK) {
-    for (int e = threadIdx.x; e < TK * TM; e += 256) {
-      const int m = e / TK, k = e % TK;
+    // all eight loads of each operand are in flight before the stores
+    float va[TK * TM / 256], vb[TK * TN / 256];
+#pragma unroll
+    for (int q = 0; q < TK * TM / 256; ++q) {
+      const int e = threadIdx.x + q * 256, m = e / TK, k = e % TK;
       const int64_t gr = row0 + m;
-      As[k][m] = (gr < rows && k0 + k < bw) ? E[gr * kBMax + k0 + k] : 0.0f;
-      const int kk = e / TN, c = e % TN;
-      const int gc = col0 + c;
-      Bs[kk][c] = (gc < n && k0 + kk < bw) ? U[static_cast<size_t>(i1 + k0 + kk) * n + gc] : 0.0f;
+      va[q] = (gr < rows && k0 + k < bw) ? __ldg(E + gr * kBMax + k0 + k) : 0.0f;
+      const int kk = e / TN, c = e % TN, gc = col0 + c;
+      vb[q] = (gc < n && k0 + kk < bw) ? __ldg(U + static_cast<size_t>(i1 + k0 + kk) * n + gc) : 0.0f;
+    }
+#pragma unroll
+    for (int q = 0; q < TK * TM / 256; ++q) {
+      const int e = threadIdx.x + q * 256;
+      As[e % TK][e / TK] = va[q];
+      Bs[e / TN][e % TN] = vb[q];
     }
     __syncthreads();
 #pragma unroll
