@@ -226,7 +226,7 @@ gptq_status gptq_quantize_layer(const void* W, gptq_dtype wdt, int64_t rows,
  * loads the library holds until the process exits.
  *   - Layers whose gptq_quantize_workspace_size(rows, n, block) exceeds
  *     GPTQ_NOALLOC_SCRATCH_BYTES are rejected with GPTQ_ERR_INVALID_ARG
- *     (e.g. 1024 x 2048 fits, 2048 x 2048 does not).
+ *     (e.g. 1024 x 1024 fits, 1024 x 2048 does not).
  *   - The first call on a device looks up the array's device address (with
  *     that device current); make that first call before any stream capture.
  *   - All calls share the array: calls whose kernels overlap on the GPU race

@@ -16,7 +16,10 @@
 //                       later columns of the block with one FMA per lane and
 //                       slot.  Group (scale, zero) are fixed when a group
 //                       starts, from the current values (warp min/max).
-//   trailing_update_kernel   W[:, i2:] -= E[:, i1:i2] * U[i1:i2, i2:] in fp32.
+//   trailing_update_tc (trailing.cu)   W[:, i2:] -= E[:, i1:i2] * U[i1:i2, i2:]
+//                       on the tensor cores, fp32-accurate through a 3-term
+//                       tf32 split; the block kernel writes E as its tf32
+//                       hi / lo halves.
 #include <algorithm>
 
 #include "common.cuh"
@@ -72,7 +75,8 @@ struct BlockArgs {
   int G;                 // group size (n when one group per row)
   int n_groups;
   float maxq;
-  float* E;              // [rows, kBMax] scaled errors of the block
+  float* E_hi;           // [rows, kBMax] scaled errors of the block, tf32 high part
+  float* E_lo;           // [rows, kBMax] and the remainder e - hi
   uint8_t* codes;        // [rows, n] processing order
   float* scales;         // [rows, n_groups]
   uint8_t* zeros;        // [rows, n_groups]
@@ -188,69 +192,13 @@ __global__ void __launch_bounds__(kRowsPerCta * 32, 1) gptq_block_kernel(BlockAr
   for (int m = 0; m < 4; ++m) {
     const int k = lane + 32 * m;
     if (k < bw) {
-      a.E[r * kBMax + k] = ek[m];
+      const float hi = __uint_as_float(__float_as_uint(ek[m]) & 0xffffe000u);
+      a.E_hi[r * kBMax + k] = hi;
+      a.E_lo[r * kBMax + k] = ek[m] - hi;
       a.codes[r * a.n + a.i1 + k] = static_cast<uint8_t>(qk[m]);
     }
   }
   if (lane == 0 && a.row_loss != nullptr) a.row_loss[r] += loss;
-}
-
-// W[:, i2:] -= E[:, 0:bw] * U[i1:i1+bw, i2:]  (fp32 SIMT, 128x128 tiles, 8x8 per thread)
-__global__ void __launch_bounds__(256) trailing_update_kernel(float* __restrict__ Wk, const float* __restrict__ E,
-                                                              const float* __restrict__ U, int64_t rows, int n,
-                                                              int i1, int bw) {
-  constexpr int TM = 128, TN = 128, TK = 16;
-  __shared__ __align__(16) float As[TK][TM];
-  __shared__ __align__(16) float Bs[TK][TN];
-  const int i2 = i1 + bw;
-  const int64_t row0 = static_cast<int64_t>(blockIdx.y) * TM;
-  const int col0 = i2 + blockIdx.x * TN;
-  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  float acc[8][8] = {};
-  for (int k0 = 0; k0 < bw; k0 += TK) {
-    // all eight loads of each operand are in flight before the stores
-    float va[TK * TM / 256], vb[TK * TN / 256];
-#pragma unroll
-    for (int q = 0; q < TK * TM / 256; ++q) {
-      const int e = threadIdx.x + q * 256, m = e / TK, k = e % TK;
-      const int64_t gr = row0 + m;
-      va[q] = (gr < rows && k0 + k < bw) ? __ldg(E + gr * kBMax + k0 + k) : 0.0f;
-      const int kk = e / TN, c = e % TN, gc = col0 + c;
-      vb[q] = (gc < n && k0 + kk < bw) ? __ldg(U + static_cast<size_t>(i1 + k0 + kk) * n + gc) : 0.0f;
-    }
-#pragma unroll
-    for (int q = 0; q < TK * TM / 256; ++q) {
-      const int e = threadIdx.x + q * 256;
-      As[e % TK][e / TK] = va[q];
-      Bs[e / TN][e % TN] = vb[q];
-    }
-    __syncthreads();
-#pragma unroll
-    for (int k = 0; k < TK; ++k) {
-      const float4 a0 = *reinterpret_cast<const float4*>(&As[k][ty * 4]);
-      const float4 a1 = *reinterpret_cast<const float4*>(&As[k][64 + ty * 4]);
-      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[k][tx * 4]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[k][64 + tx * 4]);
-      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int64_t gr = row0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + i - 4);
-    if (gr >= rows) continue;
-    float* wr = Wk + gr * n;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int gc = col0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + j - 4);
-      if (gc < n) wr[gc] -= acc[i][j];
-    }
-  }
 }
 
 // codes[r, perm[p]] = codes_p[r, p]; optional dequantized weights and g_idx.
@@ -305,18 +253,26 @@ __global__ void rtn_kernel(const T* __restrict__ W, int64_t rows, int n, int G, 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct QuantLayout {
-  size_t wk, e, codes_p, total;
+  size_t wk, e_hi, e_lo, codes_p, u_hi, u_lo, total;
+  int64_t ldu;
 };
 
 QuantLayout quant_layout(int64_t rows, int n) {
   QuantLayout l{};
+  l.ldu = (n + 3) / 4 * 4;  // 16-byte row pitch for the tensor-map loads
   size_t off = 0;
   l.wk = off;
   off += align256(static_cast<size_t>(rows) * n * sizeof(float));
-  l.e = off;
+  l.e_hi = off;
+  off += align256(static_cast<size_t>(rows) * kBMax * sizeof(float));
+  l.e_lo = off;
   off += align256(static_cast<size_t>(rows) * kBMax * sizeof(float));
   l.codes_p = off;
   off += align256(static_cast<size_t>(rows) * n);
+  l.u_hi = off;
+  off += align256(static_cast<size_t>(n) * l.ldu * sizeof(float));
+  l.u_lo = off;
+  off += align256(static_cast<size_t>(n) * l.ldu * sizeof(float));
   l.total = off;
   return l;
 }
@@ -324,6 +280,11 @@ QuantLayout quant_layout(int64_t rows, int n) {
 }  // namespace
 
 size_t quantize_workspace_size(int64_t rows, int n) { return quant_layout(rows, n).total; }
+
+gptq_status split_u_tf32(const float* U, int n, int64_t ldu, float* U_hi, float* U_lo, cudaStream_t st);
+gptq_status trailing_update_tc(float* W, int64_t ldw, int M, int N, int K, int c0, int k0, const float* E_hi,
+                               const float* E_lo, int64_t lde, const float* U_hi, const float* U_lo, int64_t ldu,
+                               int n_u, cudaStream_t st);
 
 gptq_status quantize_layer(const void* W, gptq_dtype wdt, int64_t rows, int n, const float* U, const int32_t* perm,
                            const uint8_t* dead, int bits, int group, int block, uint8_t* codes, float* scales,
@@ -333,7 +294,10 @@ gptq_status quantize_layer(const void* W, gptq_dtype wdt, int64_t rows, int n, c
   if (ws_bytes < l.total) return GPTQ_ERR_INVALID_ARG;
   uint8_t* w = static_cast<uint8_t*>(ws);
   float* Wk = reinterpret_cast<float*>(w + l.wk);
-  float* E = reinterpret_cast<float*>(w + l.e);
+  float* E_hi = reinterpret_cast<float*>(w + l.e_hi);
+  float* E_lo = reinterpret_cast<float*>(w + l.e_lo);
+  float* U_hi = reinterpret_cast<float*>(w + l.u_hi);
+  float* U_lo = reinterpret_cast<float*>(w + l.u_lo);
   uint8_t* codes_p = perm != nullptr ? w + l.codes_p : codes;
   const int G = group > 0 ? group : n;
   const int n_groups = static_cast<int>(ceil_div(n, G));
@@ -347,6 +311,7 @@ gptq_status quantize_layer(const void* W, gptq_dtype wdt, int64_t rows, int n, c
   if (row_loss != nullptr && cudaMemsetAsync(row_loss, 0, static_cast<size_t>(rows) * sizeof(float), st) != cudaSuccess)
     return GPTQ_ERR_CUDA;
   if (launch_status() != GPTQ_OK) return GPTQ_ERR_CUDA;
+  if (split_u_tf32(U, n, l.ldu, U_hi, U_lo, st) != GPTQ_OK) return GPTQ_ERR_CUDA;
 
   BlockArgs a;
   a.Wk = Wk;
@@ -356,7 +321,8 @@ gptq_status quantize_layer(const void* W, gptq_dtype wdt, int64_t rows, int n, c
   a.G = G;
   a.n_groups = n_groups;
   a.maxq = static_cast<float>((1 << bits) - 1);
-  a.E = E;
+  a.E_hi = E_hi;
+  a.E_lo = E_lo;
   a.codes = codes_p;
   a.scales = scales;
   a.zeros = zeros;
@@ -375,8 +341,9 @@ gptq_status quantize_layer(const void* W, gptq_dtype wdt, int64_t rows, int n, c
     launch(gptq_block_kernel, block_ctas, kRowsPerCta * 32, kBlockSmem, st, a);
     const int i2 = i1 + a.bw;
     if (i2 < n) {
-      const dim3 tg(static_cast<unsigned>(ceil_div(n - i2, 128)), static_cast<unsigned>(ceil_div(rows, 128)));
-      launch(trailing_update_kernel, tg, 256, 0, st, Wk, E, U, rows, n, i1, a.bw);
+      const gptq_status ts = trailing_update_tc(Wk, n, static_cast<int>(rows), n - i2, a.bw, i2, i1, E_hi, E_lo,
+                                                kBMax, U_hi, U_lo, l.ldu, n, st);
+      if (ts != GPTQ_OK) return ts;
     }
   }
   if (launch_status() != GPTQ_OK) return GPTQ_ERR_CUDA;

@@ -80,4 +80,4 @@ def test_noalloc_rejects_layers_beyond_its_scratch():
     U = torch.eye(n, device="cuda")
     st, _ = _noalloc(W, U, None, None, 4, 128, 128)
     assert st == 1  # GPTQ_ERR_INVALID_ARG
-    assert gq.LIB.gptq_quantize_workspace_size(1024, 2048, 128) <= SCRATCH_BYTES
+    assert gq.LIB.gptq_quantize_workspace_size(1024, 1024, 128) <= SCRATCH_BYTES
