@@ -8,19 +8,24 @@
 // forward through a triangular matrix.
 //
 // Per block [i1, i2) of processing positions:
-//   gptq_block_kernel   one warp per weight row; lane l holds columns
-//                       l, l+32, l+64, l+96 of the block in registers; the
-//                       block's U tile and 1/U_jj sit in shared memory.  Step
-//                       j broadcasts w_j with a shuffle, rounds it on the grid,
-//                       forms e_j = (w_j - deq_j) / U_jj and updates the
-//                       later columns of the block with one FMA per lane and
-//                       slot.  Group (scale, zero) are fixed when a group
-//                       starts, from the current values (warp min/max).
+//   gptq_block_kernel   one thread per weight row (32 rows per CTA).  The
+//                       block's 128 columns are handled as four 32-column
+//                       sub-blocks: the current sub-block lives in registers
+//                       (fully unrolled, so every index is a constant), the
+//                       rest of the block in padded shared memory.  Step j
+//                       rounds w_j on the grid, forms e_j = (w_j - deq_j) / U_jj
+//                       and updates the later columns of the sub-block; after
+//                       a sub-block its 32 errors update the later sub-blocks
+//                       from a transposed copy of the U tile.  Group (scale,
+//                       zero) come from a thread-local min/max when a group
+//                       starts.  Per row and column this costs a few
+//                       instructions instead of a warp-wide step.
 //   trailing_update_tc (trailing.cu)   W[:, i2:] -= E[:, i1:i2] * U[i1:i2, i2:]
 //                       on the tensor cores, fp32-accurate through a 3-term
 //                       tf32 split; the block kernel writes E as its tf32
 //                       hi / lo halves.
 #include <algorithm>
+#include <cstring>
 
 #include "common.cuh"
 #include "grid.cuh"
@@ -28,9 +33,11 @@
 namespace gptq {
 namespace {
 
-constexpr int kBMax = 128;       // largest block width
-constexpr int kRowsPerCta = 16;  // warps (= rows) per CTA of the block kernel
-constexpr size_t kBlockSmem = (kBMax * kBMax + kBMax) * sizeof(float);
+constexpr int kBMax = 128;        // largest block width
+constexpr int kSub = 32;          // columns of a register sub-block
+constexpr int kRowsPerCta = 32;   // rows (= threads) per CTA of the block kernel
+constexpr int kWPitch = kBMax + 1;  // shared-memory pitch of a row of the block (no bank conflicts)
+constexpr size_t kBlockSmem = (3 * kBMax * kBMax + kRowsPerCta * kWPitch + kBMax) * sizeof(float) + 16;
 
 template <typename T>
 __device__ __forceinline__ float load_w(const T* p);
@@ -72,6 +79,7 @@ struct BlockArgs {
   int64_t rows;
   int n;
   int i1, bw;            // block start and width
+  int block;             // nominal block width (the U-tile box is block x block)
   int G;                 // group size (n when one group per row)
   int n_groups;
   float maxq;
@@ -81,124 +89,247 @@ struct BlockArgs {
   float* scales;         // [rows, n_groups]
   uint8_t* zeros;        // [rows, n_groups]
   float* row_loss;       // [rows] or nullptr
+  const float2* ext_minmax;  // [rows] (min, max) of a group's columns beyond this block, or nullptr
+  int u_tma;                 // 1: the U tile arrives by TMA (u_map), 0: by plain loads
+  uint64_t wait_ns;
+  int* status;
 };
 
-__global__ void __launch_bounds__(kRowsPerCta * 32, 1) gptq_block_kernel(BlockArgs a) {
-  extern __shared__ float dyn_smem[];
-  float* us = dyn_smem;              // [kBMax][kBMax] U tile of the block
-  float* rdiag = dyn_smem + kBMax * kBMax;
+__global__ void __launch_bounds__(kRowsPerCta, 1)
+    gptq_block_kernel(const __grid_constant__ CUtensorMap u_map, const __grid_constant__ CUtensorMap uth_map,
+                      const __grid_constant__ CUtensorMap utl_map, BlockArgs a) {
+  extern __shared__ __align__(128) float dyn_smem[];
+  float* us = dyn_smem;                        // [kBMax][kBMax] U tile, us[j][k] = U[i1 + j][i1 + k]
+  float* ut = us + kBMax * kBMax;              // [kBMax][kBMax] transposed, ut[k][j] = us[j][k]
+  float* tmp = ut + kBMax * kBMax;             // [kBMax][kBMax] landing area of the transposed low half
+  float* wsm = tmp + kBMax * kBMax;            // [kRowsPerCta][kWPitch] the rows' block of weights
+  float* rdiag = wsm + kRowsPerCta * kWPitch;  // [kBMax] 1 / U_jj
+  uint64_t* bar = reinterpret_cast<uint64_t*>(rdiag + kBMax);
   const int bw = a.bw;
-  // U tile: each thread issues a batch of loads before storing any of them,
-  // 16-byte loads when the rows allow it.
-  if (bw == kBMax && a.n % 4 == 0) {
-    constexpr int kVec = kBMax * kBMax / 4 / (kRowsPerCta * 32);  // 8 float4 per thread
-    float4 v[kVec];
+  const int tid = threadIdx.x;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kRowsPerCta;
+  const int B = a.block;
+
+  // Tiles by TMA (entries past the matrix read as zero): U's block x block
+  // tile, and the same tile transposed as the two tf32 halves the trailing
+  // update uses (hi + lo == U exactly).  Without 16-byte aligned rows of U the
+  // natural tile is rebuilt from the transposed one.
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_barrier_init();
+    const uint32_t tile = static_cast<uint32_t>(B * B * sizeof(float));
+    mbar_arrive_expect_tx(bar, a.u_tma ? 3 * tile : 2 * tile);
+    if (a.u_tma) tma_load_2d(us, &u_map, bar, a.i1, a.i1);
+    tma_load_2d(ut, &uth_map, bar, a.i1, a.i1);
+    tma_load_2d(tmp, &utl_map, bar, a.i1, a.i1);
+  }
+  __syncthreads();  // the barrier is initialized before anyone waits on it
+  // the CTA's rows of the block (row rr of the tile is weight row r0 + rr),
+  // one coalesced row per load instruction, 16 rows in flight
+  const bool vec_w = (a.n % 4 == 0);
+  for (int rr0 = 0; rr0 < kRowsPerCta; rr0 += 16) {
+    float4 v[16];
 #pragma unroll
-    for (int q = 0; q < kVec; ++q) {
-      const int e = threadIdx.x + q * kRowsPerCta * 32, j = e / (kBMax / 4), k4 = e % (kBMax / 4);
-      v[q] = __ldg(reinterpret_cast<const float4*>(a.U + static_cast<size_t>(a.i1 + j) * a.n + a.i1) + k4);
-    }
-#pragma unroll
-    for (int q = 0; q < kVec; ++q) reinterpret_cast<float4*>(us)[threadIdx.x + q * kRowsPerCta * 32] = v[q];
-  } else {
-    for (int e0 = 0; e0 < kBMax * kBMax; e0 += 8 * kRowsPerCta * 32) {
-      float v[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const int e = e0 + threadIdx.x + q * kRowsPerCta * 32, j = e / kBMax, k = e % kBMax;
-        v[q] = (j < bw && k < bw) ? __ldg(a.U + static_cast<size_t>(a.i1 + j) * a.n + a.i1 + k) : 0.0f;
+    for (int q = 0; q < 16; ++q) {
+      const int64_t r = r0 + rr0 + q;
+      const int k = 4 * tid;
+      if (r < a.rows && vec_w && k + 3 < bw) {
+        v[q] = *reinterpret_cast<const float4*>(a.Wk + r * a.n + a.i1 + k);
+      } else {
+        const float* src = a.Wk + r * a.n + a.i1 + k;
+        v[q].x = (r < a.rows && k + 0 < bw) ? src[0] : 0.0f;
+        v[q].y = (r < a.rows && k + 1 < bw) ? src[1] : 0.0f;
+        v[q].z = (r < a.rows && k + 2 < bw) ? src[2] : 0.0f;
+        v[q].w = (r < a.rows && k + 3 < bw) ? src[3] : 0.0f;
       }
+    }
 #pragma unroll
-      for (int q = 0; q < 8; ++q) us[e0 + threadIdx.x + q * kRowsPerCta * 32] = v[q];
+    for (int q = 0; q < 16; ++q) {
+      float* d = wsm + (rr0 + q) * kWPitch + 4 * tid;
+      d[0] = v[q].x;
+      d[1] = v[q].y;
+      d[2] = v[q].z;
+      d[3] = v[q].w;
     }
   }
+  if (!mbar_wait(bar, 0u, a.wait_ns)) set_status(a.status, GPTQ_ERR_TIMEOUT);
   __syncthreads();
-  for (int j = threadIdx.x; j < bw; j += blockDim.x) rdiag[j] = 1.0f / us[j * kBMax + j];
-  __syncthreads();
-
-  const int lane = threadIdx.x % 32;
-  const int64_t r = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + threadIdx.x / 32;
-  if (r >= a.rows) return;
-  float* wrow = a.Wk + r * a.n;
-
-  float w[4], ek[4], qk[4];
+  // Spread the packed B x B boxes to pitch kBMax (from the last row down, so
+  // no entry is overwritten before it is read), zeroing outside the block.
+  // Rows past the block are zero already unless B < kBMax; they are written
+  // explicitly either way.
+  for (int j = kBMax - 1; j >= 0; --j) {
+    float h[kBMax / kRowsPerCta], l[kBMax / kRowsPerCta], u[kBMax / kRowsPerCta];
 #pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    const int k = lane + 32 * m;
-    w[m] = k < bw ? wrow[a.i1 + k] : 0.0f;
-    ek[m] = 0.0f;
-    qk[m] = 0.0f;
+    for (int m = 0; m < kBMax / kRowsPerCta; ++m) {  // the whole row is read ...
+      const int k = tid + m * kRowsPerCta;
+      const bool in = j < bw && k < bw;
+      h[m] = in ? ut[j * B + k] : 0.0f;
+      l[m] = in ? tmp[j * B + k] : 0.0f;
+      u[m] = in && a.u_tma ? us[j * B + k] : 0.0f;
+    }
+    __syncwarp();
+#pragma unroll
+    for (int m = 0; m < kBMax / kRowsPerCta; ++m) {  // ... before any of it is written
+      const int k = tid + m * kRowsPerCta;
+      ut[j * kBMax + k] = h[m] + l[m];
+      if (a.u_tma) us[j * kBMax + k] = u[m];
+    }
+    __syncwarp();
   }
+  __syncthreads();
+  if (!a.u_tma) {
+    for (int e = tid; e < kBMax * kBMax; e += kRowsPerCta) {
+      const int j = e / kBMax, k = e % kBMax;
+      us[e] = ut[k * kBMax + j];
+    }
+  }
+  for (int j = tid; j < kBMax; j += kRowsPerCta) rdiag[j] = j < bw ? 1.0f / ut[j * kBMax + j] : 0.0f;
+  __syncthreads();
+
+  const int64_t r = r0 + tid;
+  const bool valid = r < a.rows;
+  float* wrow = wsm + tid * kWPitch;
   // A group that began in an earlier block keeps the (scale, zero) that
   // block fixed; they are read back from the outputs.
   GridParams gp{1.0f, 0.0f};
-  if (a.i1 % a.G != 0) {
+  if (valid && a.i1 % a.G != 0) {
     const int g = a.i1 / a.G;
     gp.scale = a.scales[r * a.n_groups + g];
     gp.zero = static_cast<float>(a.zeros[r * a.n_groups + g]);
   }
   float loss = 0.0f;
+  int gpos = a.i1 % a.G;  // position of the current column inside its group
+
+  for (int sb = 0; sb * kSub < bw; ++sb) {
+    const int base = sb * kSub;
+    float w[kSub], e[kSub];
+    uint32_t cw[kSub / 4];
+#pragma unroll
+    for (int k = 0; k < kSub; ++k) w[k] = wrow[base + k];
+#pragma unroll
+    for (int k = 0; k < kSub / 4; ++k) cw[k] = 0u;
 
 #pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    if (32 * m >= bw) break;
-    for (int jj = 0; jj < 32; ++jj) {
-      const int j = 32 * m + jj;
-      if (j >= bw) break;
-      const int col = a.i1 + j;
-      if (col % a.G == 0) {
-        // Group start: (scale, zero) from the group's current values.
-        const int gend = min(col + a.G, a.n);
-        float lo = INFINITY, hi = -INFINITY;
+    for (int jj = 0; jj < kSub; ++jj) {
+      const int j = base + jj;
+      e[jj] = 0.0f;
+      if (j < bw) {
+        const int col = a.i1 + j;
+        const bool group_start = gpos == 0;
+        if (++gpos == a.G) gpos = 0;
+        if (group_start) {
+          // group start: (scale, zero) from the group's current values
+          const int gend = min(col + a.G, a.n);
+          float lo = INFINITY, hi = -INFINITY;
 #pragma unroll
-        for (int m2 = 0; m2 < 4; ++m2) {
-          const int k = lane + 32 * m2;
-          if (k >= j && k < bw && a.i1 + k < gend) {
-            lo = fminf(lo, w[m2]);
-            hi = fmaxf(hi, w[m2]);
+          for (int k = jj; k < kSub; ++k)
+            if (base + k < bw && a.i1 + base + k < gend) {
+              lo = fminf(lo, w[k]);
+              hi = fmaxf(hi, w[k]);
+            }
+          for (int k = base + kSub; k < bw && a.i1 + k < gend; ++k) {
+            lo = fminf(lo, wrow[k]);
+            hi = fmaxf(hi, wrow[k]);
+          }
+          if (valid && a.ext_minmax != nullptr && a.i1 + bw < gend) {
+            const float2 mm = a.ext_minmax[r];
+            lo = fminf(lo, mm.x);
+            hi = fmaxf(hi, mm.y);
+          }
+          gp = grid_params(lo, hi, a.maxq);
+          if (valid) {
+            const int g = col / a.G;
+            a.scales[r * a.n_groups + g] = gp.scale;
+            a.zeros[r * a.n_groups + g] = static_cast<uint8_t>(gp.zero);
           }
         }
-        for (int c = a.i1 + bw + lane; c < gend; c += 32) {
-          const float v = wrow[c];
-          lo = fminf(lo, v);
-          hi = fmaxf(hi, v);
-        }
-        lo = warp_min(lo);
-        hi = warp_max(hi);
-        gp = grid_params(lo, hi, a.maxq);
-        if (lane == 0) {
-          const int g = col / a.G;
-          a.scales[r * a.n_groups + g] = gp.scale;
-          a.zeros[r * a.n_groups + g] = static_cast<uint8_t>(gp.zero);
-        }
-      }
-      const float wj = __shfl_sync(0xffffffffu, w[m], jj);
-      const float q = grid_code(wj, gp, a.maxq);
-      const float e = __fmul_rn(__fsub_rn(wj, grid_deq(q, gp)), rdiag[j]);
-      loss = fmaf(e, e, loss);
-      if (lane == jj) {
-        ek[m] = e;
-        qk[m] = q;
-      }
-      const float* urow = us + j * kBMax;
+        const float wj = w[jj];
+        const float q = grid_code(wj, gp, a.maxq);
+        const float err = __fmul_rn(__fsub_rn(wj, grid_deq(q, gp)), rdiag[j]);
+        e[jj] = err;
+        loss = fmaf(err, err, loss);
+        cw[jj / 4] |= static_cast<uint32_t>(q) << (8 * (jj % 4));
+        // the later columns of this sub-block (U is zero outside the block)
+        const float4* urow = reinterpret_cast<const float4*>(us + j * kBMax + base);
 #pragma unroll
-      for (int m2 = 0; m2 < 4; ++m2) {
-        const int k = lane + 32 * m2;
-        if (k > j && k < bw) w[m2] = fmaf(-e, urow[k], w[m2]);
+        for (int k4 = jj / 4; k4 < kSub / 4; ++k4) {
+          const float4 u = urow[k4];
+          if (4 * k4 + 0 > jj) w[4 * k4 + 0] = fmaf(-err, u.x, w[4 * k4 + 0]);
+          if (4 * k4 + 1 > jj) w[4 * k4 + 1] = fmaf(-err, u.y, w[4 * k4 + 1]);
+          if (4 * k4 + 2 > jj) w[4 * k4 + 2] = fmaf(-err, u.z, w[4 * k4 + 2]);
+          if (4 * k4 + 3 > jj) w[4 * k4 + 3] = fmaf(-err, u.w, w[4 * k4 + 3]);
+        }
+      }
+    }
+    // the sub-block's errors update the later sub-blocks of the block, four
+    // columns at a time so the FMA chains interleave
+    for (int k = base + kSub; k < bw; k += 4) {
+      float acc[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[c] = wrow[k + c];
+#pragma unroll
+      for (int j4 = 0; j4 < kSub / 4; ++j4) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const float4 u = reinterpret_cast<const float4*>(ut + (k + c) * kBMax + base)[j4];
+          acc[c] = fmaf(-e[4 * j4 + 0], u.x, acc[c]);
+          acc[c] = fmaf(-e[4 * j4 + 1], u.y, acc[c]);
+          acc[c] = fmaf(-e[4 * j4 + 2], u.z, acc[c]);
+          acc[c] = fmaf(-e[4 * j4 + 3], u.w, acc[c]);
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) wrow[k + c] = acc[c];
+    }
+    if (valid) {
+      float* ehi = a.E_hi + r * kBMax + base;
+      float* elo = a.E_lo + r * kBMax + base;
+#pragma unroll
+      for (int k4 = 0; k4 < kSub / 4; ++k4) {
+        float4 h, l;
+        h.x = __uint_as_float(__float_as_uint(e[4 * k4 + 0]) & 0xffffe000u);
+        h.y = __uint_as_float(__float_as_uint(e[4 * k4 + 1]) & 0xffffe000u);
+        h.z = __uint_as_float(__float_as_uint(e[4 * k4 + 2]) & 0xffffe000u);
+        h.w = __uint_as_float(__float_as_uint(e[4 * k4 + 3]) & 0xffffe000u);
+        l.x = e[4 * k4 + 0] - h.x;
+        l.y = e[4 * k4 + 1] - h.y;
+        l.z = e[4 * k4 + 2] - h.z;
+        l.w = e[4 * k4 + 3] - h.w;
+        reinterpret_cast<float4*>(ehi)[k4] = h;
+        reinterpret_cast<float4*>(elo)[k4] = l;
+      }
+      uint8_t* crow = a.codes + r * a.n + a.i1 + base;
+      const int nvalid = min(kSub, bw - base);
+      if (nvalid == kSub && (reinterpret_cast<uintptr_t>(crow) % 16) == 0) {
+        reinterpret_cast<uint4*>(crow)[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        reinterpret_cast<uint4*>(crow)[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+      } else {
+#pragma unroll
+        for (int k = 0; k < kSub; ++k)
+          if (k < nvalid) crow[k] = static_cast<uint8_t>(cw[k / 4] >> (8 * (k % 4)));
       }
     }
   }
-#pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    const int k = lane + 32 * m;
-    if (k < bw) {
-      const float hi = __uint_as_float(__float_as_uint(ek[m]) & 0xffffe000u);
-      a.E_hi[r * kBMax + k] = hi;
-      a.E_lo[r * kBMax + k] = ek[m] - hi;
-      a.codes[r * a.n + a.i1 + k] = static_cast<uint8_t>(qk[m]);
-    }
+  if (valid && a.row_loss != nullptr) a.row_loss[r] += loss;
+}
+
+// Per row, (min, max) of Wk[r, c0 : c1): the part of a group that lies past
+// the block it starts in.  One warp per row.
+__global__ void group_minmax_kernel(const float* __restrict__ Wk, int64_t rows, int n, int c0, int c1,
+                                    float2* __restrict__ out) {
+  const int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
+  const int lane = threadIdx.x % 32;
+  if (r >= rows) return;
+  float lo = INFINITY, hi = -INFINITY;
+  for (int c = c0 + lane; c < c1; c += 32) {
+    const float v = Wk[r * n + c];
+    lo = fminf(lo, v);
+    hi = fmaxf(hi, v);
   }
-  if (lane == 0 && a.row_loss != nullptr) a.row_loss[r] += loss;
+  lo = warp_min(lo);
+  hi = warp_max(hi);
+  if (lane == 0) out[r] = make_float2(lo, hi);
 }
 
 // codes[r, perm[p]] = codes_p[r, p]; optional dequantized weights and g_idx.
@@ -253,7 +384,7 @@ __global__ void rtn_kernel(const T* __restrict__ W, int64_t rows, int n, int G, 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct QuantLayout {
-  size_t wk, e_hi, e_lo, codes_p, u_hi, u_lo, total;
+  size_t wk, e_hi, e_lo, codes_p, u_hi, u_lo, minmax, total;
   int64_t ldu;
 };
 
@@ -273,6 +404,8 @@ QuantLayout quant_layout(int64_t rows, int n) {
   off += align256(static_cast<size_t>(n) * l.ldu * sizeof(float));
   l.u_lo = off;
   off += align256(static_cast<size_t>(n) * l.ldu * sizeof(float));
+  l.minmax = off;
+  off += align256(static_cast<size_t>(rows) * sizeof(float2));
   l.total = off;
   return l;
 }
@@ -298,6 +431,9 @@ gptq_status quantize_layer(const void* W, gptq_dtype wdt, int64_t rows, int n, c
   float* E_lo = reinterpret_cast<float*>(w + l.e_lo);
   float* U_hi = reinterpret_cast<float*>(w + l.u_hi);
   float* U_lo = reinterpret_cast<float*>(w + l.u_lo);
+  float2* ext_minmax = reinterpret_cast<float2*>(w + l.minmax);
+  const DeviceInfo* info = device_info();
+  if (info == nullptr) return GPTQ_ERR_CUDA;
   uint8_t* codes_p = perm != nullptr ? w + l.codes_p : codes;
   const int G = group > 0 ? group : n;
   const int n_groups = static_cast<int>(ceil_div(n, G));
@@ -327,6 +463,26 @@ gptq_status quantize_layer(const void* W, gptq_dtype wdt, int64_t rows, int n, c
   a.scales = scales;
   a.zeros = zeros;
   a.row_loss = row_loss;
+  a.block = block;
+  a.wait_ns = wait_limit_ns();
+  a.status = info->status;
+  // the U tile of each block arrives as one TMA box when U's rows are
+  // 16-byte aligned
+  CUtensorMap u_map;
+  std::memset(&u_map, 0, sizeof(u_map));
+  a.u_tma = (n % 4 == 0) ? 1 : 0;
+  if (a.u_tma && !make_tensor_map_2d(&u_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, U, static_cast<uint64_t>(n),
+                                     static_cast<uint64_t>(n), static_cast<uint64_t>(n) * 4, block, block,
+                                     CU_TENSOR_MAP_SWIZZLE_NONE))
+    return GPTQ_ERR_CUDA;
+  CUtensorMap uth_map, utl_map;
+  if (!make_tensor_map_2d(&uth_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, U_hi, static_cast<uint64_t>(n),
+                          static_cast<uint64_t>(n), static_cast<uint64_t>(l.ldu) * 4, block, block,
+                          CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tensor_map_2d(&utl_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, U_lo, static_cast<uint64_t>(n),
+                          static_cast<uint64_t>(n), static_cast<uint64_t>(l.ldu) * 4, block, block,
+                          CU_TENSOR_MAP_SWIZZLE_NONE))
+    return GPTQ_ERR_CUDA;
   const unsigned block_ctas = static_cast<unsigned>(ceil_div(rows, kRowsPerCta));
   static bool attr_set = false;
   if (!attr_set) {
@@ -338,7 +494,16 @@ gptq_status quantize_layer(const void* W, gptq_dtype wdt, int64_t rows, int n, c
   for (int i1 = 0; i1 < n; i1 += block) {
     a.i1 = i1;
     a.bw = std::min(block, n - i1);
-    launch(gptq_block_kernel, block_ctas, kRowsPerCta * 32, kBlockSmem, st, a);
+    // a group that starts here and runs past the block: min / max of its
+    // columns beyond the block, taken before the block changes anything
+    const int gend = std::min(i1 + G, n);
+    a.ext_minmax = nullptr;
+    if (i1 % G == 0 && i1 + a.bw < gend) {
+      launch(group_minmax_kernel, static_cast<unsigned>(ceil_div(rows * 32, 256)), 256, 0, st, Wk, rows, n,
+             i1 + a.bw, gend, ext_minmax);
+      a.ext_minmax = ext_minmax;
+    }
+    launch(gptq_block_kernel, block_ctas, kRowsPerCta, kBlockSmem, st, u_map, uth_map, utl_map, a);
     const int i2 = i1 + a.bw;
     if (i2 < n) {
       const gptq_status ts = trailing_update_tc(Wk, n, static_cast<int>(rows), n - i2, a.bw, i2, i1, E_hi, E_lo,
