@@ -76,20 +76,26 @@ __global__ void identity_perm_kernel(int32_t* perm, int n) {
   if (i < n) perm[i] = i;
 }
 
+constexpr int kT = 64;  // tile width = panel width of the factorization below
+
 // Lower triangle of A = J P^T (H + lambda I) P J; dead diagonals become 1 + lambda.
+// Inside the kT x kT diagonal blocks the upper half is written too, as the
+// mirror of the lower one (the diagonal factorization reads whole blocks).
 __global__ void gather_reversed_kernel(const float* __restrict__ H, const int32_t* __restrict__ perm,
                                        const uint8_t* __restrict__ dead, const double* __restrict__ lambda, int n,
                                        float* __restrict__ A) {
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   const int a = blockIdx.y;
-  if (b > a || a >= n) return;
-  const int pa = perm[n - 1 - a], pb = perm[n - 1 - b];
+  if (a >= n || b >= n) return;
+  if (b > a && b / kT != a / kT) return;
+  const int lo = b > a ? a : b, hi = b > a ? b : a;  // the lower-triangle entry (hi, lo) holds the value
+  const int ph = perm[n - 1 - hi], pl = perm[n - 1 - lo];
   float v;
   if (a == b) {
-    const double base = dead[pa] ? 1.0 : static_cast<double>(H[static_cast<size_t>(pa) * n + pa]);
+    const double base = dead[ph] ? 1.0 : static_cast<double>(H[static_cast<size_t>(ph) * n + ph]);
     v = static_cast<float>(base + *lambda);
   } else {
-    v = H[static_cast<size_t>(pa) * n + pb];
+    v = H[static_cast<size_t>(ph) * n + pl];
   }
   A[static_cast<size_t>(a) * n + b] = v;
 }
@@ -114,7 +120,6 @@ __global__ void gather_reversed_kernel(const float* __restrict__ H, const int32_
 // into U's rotated position (U = J X J), so no rotation pass is needed;
 // R's tiles live in the same places before they are finalized.
 
-constexpr int kT = 64;             // tile width = panel width
 constexpr int kPad = 68;           // shared-memory row stride (16-byte aligned rows)
 constexpr int kCholThreads = 256;
 constexpr size_t kCholSmem = 3 * kT * kPad * sizeof(float);
@@ -165,142 +170,93 @@ __device__ __forceinline__ void tile_product(const Tile* P, const Tile* Q, float
   }
 }
 
-// Lower Cholesky of the 16 x 16 block of `a` at (o, o) by one warp (lanes
-// 0..15 own its rows), shuffles only; then the block's inverse, lane c
-// solving L x = e_c for column c.  The loops have constant trip counts and
-// predicated bodies so that they unroll completely and the row / column stay
-// in registers (this kernel runs at its register limit).
-__device__ __forceinline__ void warp_chol_inv16(Tile* a, Tile* inv, int o, int* fstatus) {
-  const int lane = threadIdx.x & 31;
-  const int row = lane & 15;
-  float r[16];
-#pragma unroll
-  for (int c = 0; c < 16; ++c) r[c] = a[o + row][o + c];
-#pragma unroll 16
-  for (int j = 0; j < 16; ++j) {
-    float piv = __shfl_sync(0xffffffffu, r[j], j);
-    if (!(piv > 0.0f) || !isfinite(piv)) {
-      if (lane == 0) set_status(fstatus, isfinite(piv) ? GPTQ_ERR_NOT_PD : GPTQ_ERR_NONFINITE);
-      piv = 1.0f;
-    }
-    const float d = sqrtf(piv);
-    const float rd = 1.0f / d;
-    const float l = row > j ? r[j] * rd : (row == j ? d : 0.0f);
-    r[j] = l;
-#pragma unroll 16
-    for (int c = 0; c < 16; ++c) {
-      const float lc = __shfl_sync(0xffffffffu, l, c);
-      if (c > j && row >= c) r[c] = fmaf(-l, lc, r[c]);
-    }
-  }
-  if (lane < 16) {
-#pragma unroll
-    for (int c = 0; c < 16; ++c) a[o + row][o + c] = c <= row ? r[c] : 0.0f;
-  }
-  __syncwarp();
-  float x[16];
-#pragma unroll 16
-  for (int q = 0; q < 16; ++q) {
-    float s = q == row ? 1.0f : 0.0f;
-#pragma unroll 16
-    for (int m = 0; m < 16; ++m)
-      if (m < q) s = fmaf(-a[o + q][o + m], x[m], s);
-    x[q] = q >= row ? s / a[o + q][o + q] : 0.0f;
-  }
-  if (lane < 16) {
-#pragma unroll
-    for (int q = 0; q < 16; ++q) inv[o + q][o + row] = x[q];
-  }
-}
-
 // Factors the diagonal block k: L_kk into A, Linv_kk into X's diagonal tile.
-// One CTA.  Four 16-wide block columns: a warp factors and inverts the 16 x 16
-// diagonal piece, the CTA solves the piece below it and updates the trailing
-// part; then the inverse's off-diagonal pieces follow by block forward
-// substitution, X_ij = -X_ii sum_{m=j}^{i-1} L_im X_mj.
-__device__ void factor_diag(const CholArgs& p, int k, Tile* a, Tile* inv, Tile* t) {
+//
+// A right-looking sweep over the block's 64 pivots by the whole CTA, with the
+// inverse built in the same sweep (R = I; at pivot j, X_j = R_j / L_jj and
+// R_i -= L_ij X_j for i > j).  Thread t holds row i = t / 4, columns
+// 16 (t % 4) .. 16 (t % 4) + 15 of the block in registers: left of the pivot
+// those are R's entries, right of it the remaining matrix, upper half
+// included.  The upper half makes row j carry, by symmetry, the column under
+// the pivot too, so one broadcast per pivot suffices: the four threads of row
+// j + 1 store their registers to shared memory (R_{j+1,<j+1}, the next pivot,
+// and A_{j+1,>j+1}), one barrier, and every thread reads the pivot, its own
+// row's multiplier and its sixteen columns from there.  With s_i = A_ij / d_j
+// (d_j the pivot), every update is v -= s_i * row_j[c]: the Schur update
+// A_ic -= L_ij L_cj on the right of the pivot and R_ic -= L_ij X_jc on its
+// left; the pivot column itself becomes R_ij = -s_i.  X's rows are scaled by
+// 1 / L_ii at the end.  A pivot that is not positive or not finite sets the
+// status word (a non-finite one takes precedence) and is replaced by 1.
+__device__ void factor_diag(const CholArgs& p, int k, Tile* lout, Tile* xout, Tile* bt) {
   const int k0 = k * kT;
   const int kb = min(kT, p.n - k0);
-  {
-    float v[kPerThread];
+  const int t = threadIdx.x, i = t >> 2, q = t & 3;
+  float* bbuf = &bt[0][0];  // two 64-float broadcast rows (pivot parity)
+  float v[16];
 #pragma unroll
-    for (int q = 0; q < kPerThread; ++q) {
-      const int e = threadIdx.x + q * kCholThreads, r = e / kT, c = e % kT;
-      v[q] = (r < kb && c <= r) ? ld_a(p, k0 + r, k0 + c) : (r == c ? 1.0f : 0.0f);
-    }
+  for (int m = 0; m < 16; ++m) {
+    const int c = 16 * q + m;
+    v[m] = (i < kb && c < kb) ? ld_a(p, k0 + i, k0 + c) : (i == c ? 1.0f : 0.0f);
+  }
+  if (i == 0) {
+    float4* d4 = reinterpret_cast<float4*>(bbuf + 16 * q);
 #pragma unroll
-    for (int q = 0; q < kPerThread; ++q) {
-      const int e = threadIdx.x + q * kCholThreads, r = e / kT, c = e % kT;
-      a[r][c] = v[q];
-      inv[r][c] = 0.0f;
-    }
+    for (int g = 0; g < 4; ++g) d4[g] = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
   }
   __syncthreads();
-  const int warp = threadIdx.x / 32;
-  for (int kk = 0; kk < 4; ++kk) {
-    const int o = 16 * kk;
-    if (warp == 0) warp_chol_inv16(a, inv, o, p.fstatus);
-    __syncthreads();
-    const int below = kT - o - 16;
-    if (below > 0) {
-      // L_below = A_below * Linv_oo^T  (below x 16), 3 values per thread at most
-      float v[3];
+  float myrd = 1.0f;
+  bool notpd = false, nonfinite = false;
+#pragma unroll 1
+  for (int j0 = 0; j0 < kT; j0 += 16) {
+    // sixteen pivots per iteration, unrolled so that register indices are constants
 #pragma unroll
-      for (int q = 0; q < 3; ++q) {
-        const int e = threadIdx.x + q * kCholThreads;
-        float s = 0.0f;
-        if (e < below * 16) {
-          const int r = o + 16 + e / 16, c = e % 16;
-          for (int d = 0; d <= c; ++d) s = fmaf(a[r][o + d], inv[o + c][o + d], s);
-        }
-        v[q] = s;
+    for (int jj = 0; jj < 16; ++jj) {
+      const int j = j0 + jj;
+      const float* B = bbuf + (j & 1) * kT;
+      float* Bn = bbuf + ((j + 1) & 1) * kT;
+      float d = B[j];
+      const float bi = B[i];
+      float bc[16];
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const float4 w = *reinterpret_cast<const float4*>(B + 16 * q + 4 * g);
+        bc[4 * g] = w.x;
+        bc[4 * g + 1] = w.y;
+        bc[4 * g + 2] = w.z;
+        bc[4 * g + 3] = w.w;
       }
-      __syncthreads();
+      nonfinite |= !isfinite(d);
+      notpd |= !(d > 0.0f);
+      d = (d > 0.0f && d < INFINITY) ? d : 1.0f;
+      const float rd = rsqrtf(d);
+      const float s = bi * rd * rd;
+      if (i > j) {
 #pragma unroll
-      for (int q = 0; q < 3; ++q) {
-        const int e = threadIdx.x + q * kCholThreads;
-        if (e < below * 16) a[o + 16 + e / 16][o + e % 16] = v[q];
+        for (int m = 0; m < 16; ++m) v[m] = fmaf(-s, bc[m], v[m]);
+        if (q == (j0 >> 4)) v[jj] = -s;
       }
-      __syncthreads();
-      // trailing update of the lower part below the block column
-      for (int e = threadIdx.x; e < below * below; e += kCholThreads) {
-        const int r = o + 16 + e / below, c = o + 16 + e % below;
-        if (c <= r) {
-          float s = 0.0f;
+      myrd = i == j ? rd : myrd;
+      if (q == 0 && i >= j) lout[i][j] = (i == j ? d : bi) * rd;
+      if (i == j + 1) {
+        float4* d4 = reinterpret_cast<float4*>(Bn + 16 * q);
 #pragma unroll
-          for (int d = 0; d < 16; ++d) s = fmaf(a[r][o + d], a[c][o + d], s);
-          a[r][c] -= s;
-        }
+        for (int g = 0; g < 4; ++g) d4[g] = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
       }
       __syncthreads();
     }
   }
-  // off-diagonal pieces of the inverse, block row by block row
-  for (int bi = 1; bi < 4; ++bi) {
-    const int ri = 16 * bi;
-    // t[r][c] = sum_{m=j}^{bi-1} L[ri + r][16 m ..] X[16 m .., c], for c < ri
-    for (int e = threadIdx.x; e < 16 * ri; e += kCholThreads) {
-      const int r = e / ri, c = e % ri;
-      const int j = c / 16;
-      float s = 0.0f;
-      for (int d = 16 * j; d < ri; ++d) s = fmaf(a[ri + r][d], inv[d][c], s);
-      t[r][c] = s;
-    }
-    __syncthreads();
-    for (int e = threadIdx.x; e < 16 * ri; e += kCholThreads) {
-      const int r = e / ri, c = e % ri;
-      float s = 0.0f;
+  if (t == 0 && (nonfinite || notpd)) set_status(p.fstatus, nonfinite ? GPTQ_ERR_NONFINITE : GPTQ_ERR_NOT_PD);
 #pragma unroll
-      for (int d = 0; d < 16; ++d) s = fmaf(inv[ri + r][ri + d], t[d][c], s);
-      inv[ri + r][c] = -s;
-    }
-    __syncthreads();
+  for (int m = 0; m < 16; ++m) {
+    const int c = 16 * q + m;
+    xout[i][c] = c < i ? v[m] * myrd : (c == i ? myrd : 0.0f);
   }
+  __syncthreads();
   for (int e = threadIdx.x; e < kT * kT; e += kCholThreads) {
     const int r = e / kT, c = e % kT;
     if (r < kb && c < kb) {
-      if (c <= r) *at_a(p, k0 + r, k0 + c) = a[r][c];
-      *at_x(p, k0 + r, k0 + c) = inv[r][c];
+      if (c <= r) *at_a(p, k0 + r, k0 + c) = lout[r][c];
+      *at_x(p, k0 + r, k0 + c) = xout[r][c];
     }
   }
   __syncthreads();
