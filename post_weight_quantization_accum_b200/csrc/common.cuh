@@ -79,6 +79,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
 }
 
 // ---------------------------------------------------------------------------
+// 4-byte asynchronous global -> shared copy; src_bytes = 0 writes a zero
+// instead of reading (cp.async with a source size).
+__device__ __forceinline__ void cp_async_4(void* smem_dst, const void* gmem_src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(smem_u32(smem_dst)), "l"(gmem_src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
+
 // TMA (cp.async.bulk.tensor), no multicast
 // ---------------------------------------------------------------------------
 

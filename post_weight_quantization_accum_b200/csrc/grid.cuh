@@ -36,6 +36,22 @@ __device__ __forceinline__ float grid_code(float w, GridParams p, float maxq) {
   return fminf(fmaxf(q, 0.0f), maxq);
 }
 
+// grid_code with the division replaced by a product with rcp = 1 / scale
+// (correctly rounded), and the quotient formed only where that could change
+// the code.  rcp and the product each round once, so t = w * rcp lies within
+// 3 * 2^-24 * |w / scale| of the correctly rounded quotient; rint(t) is the
+// quotient's rint unless a half-integer lies within that distance of t.  The
+// test below uses 2^-21 * |t| and also sends |t| >= 2^22 and non-finite t
+// (a subnormal scale) to the exact quotient, so the code is grid_code's.
+__device__ __forceinline__ float grid_code_rcp(float w, GridParams p, float rcp, float maxq) {
+  const float t = __fmul_rn(w, rcp);
+  float k = rintf(t);
+  const float to_half = fabsf(__fsub_rn(fabsf(__fsub_rn(t, k)), 0.5f));
+  if (!(fabsf(t) < 4194304.0f) || to_half <= 4.76837158e-7f * fabsf(t)) k = rintf(__fdiv_rn(w, p.scale));
+  const float q = __fadd_rn(k, p.zero);
+  return fminf(fmaxf(q, 0.0f), maxq);
+}
+
 // Dequantized value scale * (code - zero).
 __device__ __forceinline__ float grid_deq(float code, GridParams p) {
   return __fmul_rn(p.scale, __fsub_rn(code, p.zero));

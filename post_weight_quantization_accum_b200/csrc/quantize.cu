@@ -8,18 +8,20 @@
 // forward through a triangular matrix.
 //
 // Per block [i1, i2) of processing positions:
-//   gptq_block_kernel   one thread per weight row (32 rows per CTA).  The
-//                       block's 128 columns are handled as four 32-column
-//                       sub-blocks: the current sub-block lives in registers
-//                       (fully unrolled, so every index is a constant), the
-//                       rest of the block in padded shared memory.  Step j
-//                       rounds w_j on the grid, forms e_j = (w_j - deq_j) / U_jj
-//                       and updates the later columns of the sub-block; after
-//                       a sub-block its 32 errors update the later sub-blocks
-//                       from a transposed copy of the U tile.  Group (scale,
-//                       zero) come from a thread-local min/max when a group
-//                       starts.  Per row and column this costs a few
-//                       instructions instead of a warp-wide step.
+//   gptq_block_kernel   sixteen lanes per weight row (two rows per warp),
+//                       lane l owning the block's columns l, l + 16, ...,
+//                       l + 112 in registers, the block's U tile in shared
+//                       memory (each lane's eight entries of a U row side by
+//                       side, two vector loads per step).  Step j broadcasts
+//                       w_j from its owner lane (shuffle), every lane rounds
+//                       it on the grid and forms e_j = (w_j - deq_j) / U_jj,
+//                       then updates its own columns w_k -= e_j U_jk (U is
+//                       zero left of the diagonal, so no lane needs a test).
+//                       Group (scale, zero) are a shuffle min / max reduction
+//                       over the group's current values when the group
+//                       starts.  No block-wide synchronisation inside the
+//                       loop; one row's chain of dependent steps overlaps the
+//                       other warps'.
 //   trailing_update_tc (trailing.cu)   W[:, i2:] -= E[:, i1:i2] * U[i1:i2, i2:]
 //                       on the tensor cores, fp32-accurate through a 3-term
 //                       tf32 split; the block kernel writes E as its tf32
@@ -34,10 +36,8 @@ namespace gptq {
 namespace {
 
 constexpr int kBMax = 128;        // largest block width
-constexpr int kSub = 32;          // columns of a register sub-block
-constexpr int kRowsPerCta = 32;   // rows (= threads) per CTA of the block kernel
-constexpr int kWPitch = kBMax + 1;  // shared-memory pitch of a row of the block (no bank conflicts)
-constexpr size_t kBlockSmem = (3 * kBMax * kBMax + kRowsPerCta * kWPitch + kBMax) * sizeof(float) + 16;
+constexpr int kMaxWarpsPerCta = 32;
+constexpr int kBlockLanes = 16;  // lanes per weight row in the block kernel
 
 template <typename T>
 __device__ __forceinline__ float load_w(const T* p);
@@ -79,239 +79,158 @@ struct BlockArgs {
   int64_t rows;
   int n;
   int i1, bw;            // block start and width
-  int block;             // nominal block width (the U-tile box is block x block)
   int G;                 // group size (n when one group per row)
   int n_groups;
   float maxq;
-  float* E_hi;           // [rows, kBMax] scaled errors of the block, tf32 high part
-  float* E_lo;           // [rows, kBMax] and the remainder e - hi
+  float* E_hi;           // [rows, lde] scaled errors, tf32 high part (this block at column e_off)
+  float* E_lo;           // [rows, lde] and the remainder e - hi
+  int lde, e_off;
   uint8_t* codes;        // [rows, n] processing order
   float* scales;         // [rows, n_groups]
   uint8_t* zeros;        // [rows, n_groups]
   float* row_loss;       // [rows] or nullptr
   const float2* ext_minmax;  // [rows] (min, max) of a group's columns beyond this block, or nullptr
-  int u_tma;                 // 1: the U tile arrives by TMA (u_map), 0: by plain loads
-  uint64_t wait_ns;
-  int* status;
 };
 
-__global__ void __launch_bounds__(kRowsPerCta, 1)
-    gptq_block_kernel(const __grid_constant__ CUtensorMap u_map, const __grid_constant__ CUtensorMap uth_map,
-                      const __grid_constant__ CUtensorMap utl_map, BlockArgs a) {
-  extern __shared__ __align__(128) float dyn_smem[];
-  float* us = dyn_smem;                        // [kBMax][kBMax] U tile, us[j][k] = U[i1 + j][i1 + k]
-  float* ut = us + kBMax * kBMax;              // [kBMax][kBMax] transposed, ut[k][j] = us[j][k]
-  float* tmp = ut + kBMax * kBMax;             // [kBMax][kBMax] landing area of the transposed low half
-  float* wsm = tmp + kBMax * kBMax;            // [kRowsPerCta][kWPitch] the rows' block of weights
-  float* rdiag = wsm + kRowsPerCta * kWPitch;  // [kBMax] 1 / U_jj
-  uint64_t* bar = reinterpret_cast<uint64_t*>(rdiag + kBMax);
+// Lanes per weight row and the shared-memory layout of the U tile: lane li of
+// a row owns the block columns li + kLanes m (m < kBMax / kLanes), and row j
+// of the tile keeps each lane's entries side by side at a stride of
+// kLanes * pitch with a lane pitch whose multiples fall in distinct 16-byte
+// bank groups (so the vector loads of eight consecutive lanes do not conflict).
+template <int kLanes>
+struct BlockShape {
+  static constexpr int kCols = kBMax / kLanes;                // columns per lane
+  static constexpr int kPitch = kCols == 4 ? 4 : kCols + 4;   // floats per lane slot
+  static constexpr int kRowPitch = kLanes * kPitch;           // floats per tile row
+  static constexpr size_t kSmem = (static_cast<size_t>(kBMax) * kRowPitch + kBMax) * sizeof(float);
+};
+
+template <int kLanes>
+__global__ void __launch_bounds__(kMaxWarpsPerCta * 32, 1) gptq_block_kernel(BlockArgs a) {
+  using Shape = BlockShape<kLanes>;
+  constexpr int C = Shape::kCols;
+  extern __shared__ __align__(16) float dyn_smem[];
+  float* us = dyn_smem;                             // [kBMax][kRowPitch] the U tile, lane-major
+  float* rdiag = us + kBMax * Shape::kRowPitch;     // [kBMax] 1 / U_jj
   const int bw = a.bw;
-  const int tid = threadIdx.x;
-  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kRowsPerCta;
-  const int B = a.block;
-
-  // Tiles by TMA (entries past the matrix read as zero): U's block x block
-  // tile, and the same tile transposed as the two tf32 halves the trailing
-  // update uses (hi + lo == U exactly).  Without 16-byte aligned rows of U the
-  // natural tile is rebuilt from the transposed one.
-  if (tid == 0) {
-    mbar_init(bar, 1);
-    fence_barrier_init();
-    const uint32_t tile = static_cast<uint32_t>(B * B * sizeof(float));
-    mbar_arrive_expect_tx(bar, a.u_tma ? 3 * tile : 2 * tile);
-    if (a.u_tma) tma_load_2d(us, &u_map, bar, a.i1, a.i1);
-    tma_load_2d(ut, &uth_map, bar, a.i1, a.i1);
-    tma_load_2d(tmp, &utl_map, bar, a.i1, a.i1);
+  const int lane = threadIdx.x & 31;
+  const int li = lane % kLanes;  // lane within its row group
+  const int warps = blockDim.x >> 5;
+  // the tile by asynchronous 4-byte copies, all in flight at once, scattered
+  // to the lane-major layout (coalesced along U's rows; zeros outside the block)
+  for (int e = threadIdx.x; e < kBMax * kBMax; e += blockDim.x) {
+    const int j = e / kBMax, c = e % kBMax;
+    const bool in = j < bw && c < bw;
+    const float* src = in ? a.U + static_cast<int64_t>(a.i1 + j) * a.n + a.i1 + c : a.U;
+    cp_async_4(us + j * Shape::kRowPitch + (c % kLanes) * Shape::kPitch + c / kLanes, src, in ? 4u : 0u);
   }
-  __syncthreads();  // the barrier is initialized before anyone waits on it
-  // the CTA's rows of the block (row rr of the tile is weight row r0 + rr),
-  // one coalesced row per load instruction, 16 rows in flight
-  const bool vec_w = (a.n % 4 == 0);
-  for (int rr0 = 0; rr0 < kRowsPerCta; rr0 += 16) {
-    float4 v[16];
-#pragma unroll
-    for (int q = 0; q < 16; ++q) {
-      const int64_t r = r0 + rr0 + q;
-      const int k = 4 * tid;
-      if (r < a.rows && vec_w && k + 3 < bw) {
-        v[q] = *reinterpret_cast<const float4*>(a.Wk + r * a.n + a.i1 + k);
-      } else {
-        const float* src = a.Wk + r * a.n + a.i1 + k;
-        v[q].x = (r < a.rows && k + 0 < bw) ? src[0] : 0.0f;
-        v[q].y = (r < a.rows && k + 1 < bw) ? src[1] : 0.0f;
-        v[q].z = (r < a.rows && k + 2 < bw) ? src[2] : 0.0f;
-        v[q].w = (r < a.rows && k + 3 < bw) ? src[3] : 0.0f;
-      }
-    }
-#pragma unroll
-    for (int q = 0; q < 16; ++q) {
-      float* d = wsm + (rr0 + q) * kWPitch + 4 * tid;
-      d[0] = v[q].x;
-      d[1] = v[q].y;
-      d[2] = v[q].z;
-      d[3] = v[q].w;
-    }
-  }
-  if (!mbar_wait(bar, 0u, a.wait_ns)) set_status(a.status, GPTQ_ERR_TIMEOUT);
+  cp_async_wait_all();
   __syncthreads();
-  // Spread the packed B x B boxes to pitch kBMax (from the last row down, so
-  // no entry is overwritten before it is read), zeroing outside the block.
-  // Rows past the block are zero already unless B < kBMax; they are written
-  // explicitly either way.
-  for (int j = kBMax - 1; j >= 0; --j) {
-    float h[kBMax / kRowsPerCta], l[kBMax / kRowsPerCta], u[kBMax / kRowsPerCta];
-#pragma unroll
-    for (int m = 0; m < kBMax / kRowsPerCta; ++m) {  // the whole row is read ...
-      const int k = tid + m * kRowsPerCta;
-      const bool in = j < bw && k < bw;
-      h[m] = in ? ut[j * B + k] : 0.0f;
-      l[m] = in ? tmp[j * B + k] : 0.0f;
-      u[m] = in && a.u_tma ? us[j * B + k] : 0.0f;
-    }
-    __syncwarp();
-#pragma unroll
-    for (int m = 0; m < kBMax / kRowsPerCta; ++m) {  // ... before any of it is written
-      const int k = tid + m * kRowsPerCta;
-      ut[j * kBMax + k] = h[m] + l[m];
-      if (a.u_tma) us[j * kBMax + k] = u[m];
-    }
-    __syncwarp();
-  }
-  __syncthreads();
-  if (!a.u_tma) {
-    for (int e = tid; e < kBMax * kBMax; e += kRowsPerCta) {
-      const int j = e / kBMax, k = e % kBMax;
-      us[e] = ut[k * kBMax + j];
-    }
-  }
-  for (int j = tid; j < kBMax; j += kRowsPerCta) rdiag[j] = j < bw ? 1.0f / ut[j * kBMax + j] : 0.0f;
+  for (int j = threadIdx.x; j < kBMax; j += blockDim.x)
+    rdiag[j] = j < bw ? 1.0f / us[j * Shape::kRowPitch + (j % kLanes) * Shape::kPitch + j / kLanes] : 0.0f;
   __syncthreads();
 
-  const int64_t r = r0 + tid;
-  const bool valid = r < a.rows;
-  float* wrow = wsm + tid * kWPitch;
+  const int64_t warp_row0 = (static_cast<int64_t>(blockIdx.x) * warps + (threadIdx.x >> 5)) * (32 / kLanes);
+  if (warp_row0 >= a.rows) return;  // whole warps leave; no block-wide barrier follows
+  const int64_t r = warp_row0 + lane / kLanes;
+  const bool valid = r < a.rows;    // a warp's last rows may lie past the matrix
+  const int64_t rr = valid ? r : a.rows - 1;  // such lanes compute on a real row and write nothing
+  const float* wsrc = a.Wk + rr * a.n + a.i1;
+  float w[C];
+#pragma unroll
+  for (int m = 0; m < C; ++m) {
+    const int c = li + kLanes * m;
+    w[m] = c < bw ? wsrc[c] : 0.0f;
+  }
   // A group that began in an earlier block keeps the (scale, zero) that
   // block fixed; they are read back from the outputs.
   GridParams gp{1.0f, 0.0f};
-  if (valid && a.i1 % a.G != 0) {
+  if (a.i1 % a.G != 0) {
     const int g = a.i1 / a.G;
-    gp.scale = a.scales[r * a.n_groups + g];
-    gp.zero = static_cast<float>(a.zeros[r * a.n_groups + g]);
+    gp.scale = a.scales[rr * a.n_groups + g];
+    gp.zero = static_cast<float>(a.zeros[rr * a.n_groups + g]);
   }
+  float rcp = __frcp_rn(gp.scale);
   float loss = 0.0f;
-  int gpos = a.i1 % a.G;  // position of the current column inside its group
-
-  for (int sb = 0; sb * kSub < bw; ++sb) {
-    const int base = sb * kSub;
-    float w[kSub], e[kSub];
-    uint32_t cw[kSub / 4];
+  float e_own[C], q_own[C];  // this lane's columns' errors and codes
 #pragma unroll
-    for (int k = 0; k < kSub; ++k) w[k] = wrow[base + k];
-#pragma unroll
-    for (int k = 0; k < kSub / 4; ++k) cw[k] = 0u;
+  for (int m = 0; m < C; ++m) e_own[m] = q_own[m] = 0.0f;
+  int jg = (a.G - a.i1 % a.G) % a.G;  // block position of the next group start
+  const float* ulane = us + li * Shape::kPitch;
 
 #pragma unroll
-    for (int jj = 0; jj < kSub; ++jj) {
-      const int j = base + jj;
-      e[jj] = 0.0f;
-      if (j < bw) {
-        const int col = a.i1 + j;
-        const bool group_start = gpos == 0;
-        if (++gpos == a.G) gpos = 0;
-        if (group_start) {
-          // group start: (scale, zero) from the group's current values
-          const int gend = min(col + a.G, a.n);
-          float lo = INFINITY, hi = -INFINITY;
+  for (int mj = 0; mj < C; ++mj) {
+    const int jend = min(kLanes, bw - kLanes * mj);
+#pragma unroll 1
+    for (int jj = 0; jj < jend; ++jj) {
+      const int j = kLanes * mj + jj;
+      if (j == jg) {
+        // group start: (scale, zero) from the group's current values
+        jg += a.G;
+        const int gend = min(a.i1 + j + a.G, a.n);
+        float lo = INFINITY, hi = -INFINITY;
 #pragma unroll
-          for (int k = jj; k < kSub; ++k)
-            if (base + k < bw && a.i1 + base + k < gend) {
-              lo = fminf(lo, w[k]);
-              hi = fmaxf(hi, w[k]);
-            }
-          for (int k = base + kSub; k < bw && a.i1 + k < gend; ++k) {
-            lo = fminf(lo, wrow[k]);
-            hi = fmaxf(hi, wrow[k]);
-          }
-          if (valid && a.ext_minmax != nullptr && a.i1 + bw < gend) {
-            const float2 mm = a.ext_minmax[r];
-            lo = fminf(lo, mm.x);
-            hi = fmaxf(hi, mm.y);
-          }
-          gp = grid_params(lo, hi, a.maxq);
-          if (valid) {
-            const int g = col / a.G;
-            a.scales[r * a.n_groups + g] = gp.scale;
-            a.zeros[r * a.n_groups + g] = static_cast<uint8_t>(gp.zero);
+        for (int m = 0; m < C; ++m) {
+          const int c = li + kLanes * m;
+          if (c >= j && c < bw && a.i1 + c < gend) {
+            lo = fminf(lo, w[m]);
+            hi = fmaxf(hi, w[m]);
           }
         }
-        const float wj = w[jj];
-        const float q = grid_code(wj, gp, a.maxq);
-        const float err = __fmul_rn(__fsub_rn(wj, grid_deq(q, gp)), rdiag[j]);
-        e[jj] = err;
-        loss = fmaf(err, err, loss);
-        cw[jj / 4] |= static_cast<uint32_t>(q) << (8 * (jj % 4));
-        // the later columns of this sub-block (U is zero outside the block)
-        const float4* urow = reinterpret_cast<const float4*>(us + j * kBMax + base);
 #pragma unroll
-        for (int k4 = jj / 4; k4 < kSub / 4; ++k4) {
-          const float4 u = urow[k4];
-          if (4 * k4 + 0 > jj) w[4 * k4 + 0] = fmaf(-err, u.x, w[4 * k4 + 0]);
-          if (4 * k4 + 1 > jj) w[4 * k4 + 1] = fmaf(-err, u.y, w[4 * k4 + 1]);
-          if (4 * k4 + 2 > jj) w[4 * k4 + 2] = fmaf(-err, u.z, w[4 * k4 + 2]);
-          if (4 * k4 + 3 > jj) w[4 * k4 + 3] = fmaf(-err, u.w, w[4 * k4 + 3]);
+        for (int o = kLanes / 2; o > 0; o >>= 1) {
+          lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+          hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+        }
+        if (a.ext_minmax != nullptr && a.i1 + bw < gend) {
+          const float2 mm = a.ext_minmax[rr];
+          lo = fminf(lo, mm.x);
+          hi = fmaxf(hi, mm.y);
+        }
+        gp = grid_params(lo, hi, a.maxq);
+        rcp = __frcp_rn(gp.scale);
+        if (li == 0 && valid) {
+          const int g = (a.i1 + j) / a.G;
+          a.scales[r * a.n_groups + g] = gp.scale;
+          a.zeros[r * a.n_groups + g] = static_cast<uint8_t>(gp.zero);
         }
       }
-    }
-    // the sub-block's errors update the later sub-blocks of the block, four
-    // columns at a time so the FMA chains interleave
-    for (int k = base + kSub; k < bw; k += 4) {
-      float acc[4];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) acc[c] = wrow[k + c];
-#pragma unroll
-      for (int j4 = 0; j4 < kSub / 4; ++j4) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const float4 u = reinterpret_cast<const float4*>(ut + (k + c) * kBMax + base)[j4];
-          acc[c] = fmaf(-e[4 * j4 + 0], u.x, acc[c]);
-          acc[c] = fmaf(-e[4 * j4 + 1], u.y, acc[c]);
-          acc[c] = fmaf(-e[4 * j4 + 2], u.z, acc[c]);
-          acc[c] = fmaf(-e[4 * j4 + 3], u.w, acc[c]);
-        }
+      const float wj = __shfl_sync(0xffffffffu, w[mj], jj, kLanes);
+      const float q = grid_code_rcp(wj, gp, rcp, a.maxq);
+      const float err = __fmul_rn(__fsub_rn(wj, grid_deq(q, gp)), rdiag[j]);
+      loss = fmaf(err, err, loss);
+      if (li == jj) {
+        e_own[mj] = err;
+        q_own[mj] = q;
       }
+      // w_k -= e_j U_jk for this lane's columns (U_jk = 0 for k < j; the
+      // column j itself is not read again)
+      const float4* urow = reinterpret_cast<const float4*>(ulane + j * Shape::kRowPitch);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) wrow[k + c] = acc[c];
-    }
-    if (valid) {
-      float* ehi = a.E_hi + r * kBMax + base;
-      float* elo = a.E_lo + r * kBMax + base;
-#pragma unroll
-      for (int k4 = 0; k4 < kSub / 4; ++k4) {
-        float4 h, l;
-        h.x = __uint_as_float(__float_as_uint(e[4 * k4 + 0]) & 0xffffe000u);
-        h.y = __uint_as_float(__float_as_uint(e[4 * k4 + 1]) & 0xffffe000u);
-        h.z = __uint_as_float(__float_as_uint(e[4 * k4 + 2]) & 0xffffe000u);
-        h.w = __uint_as_float(__float_as_uint(e[4 * k4 + 3]) & 0xffffe000u);
-        l.x = e[4 * k4 + 0] - h.x;
-        l.y = e[4 * k4 + 1] - h.y;
-        l.z = e[4 * k4 + 2] - h.z;
-        l.w = e[4 * k4 + 3] - h.w;
-        reinterpret_cast<float4*>(ehi)[k4] = h;
-        reinterpret_cast<float4*>(elo)[k4] = l;
-      }
-      uint8_t* crow = a.codes + r * a.n + a.i1 + base;
-      const int nvalid = min(kSub, bw - base);
-      if (nvalid == kSub && (reinterpret_cast<uintptr_t>(crow) % 16) == 0) {
-        reinterpret_cast<uint4*>(crow)[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-        reinterpret_cast<uint4*>(crow)[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
-      } else {
-#pragma unroll
-        for (int k = 0; k < kSub; ++k)
-          if (k < nvalid) crow[k] = static_cast<uint8_t>(cw[k / 4] >> (8 * (k % 4)));
+      for (int g4 = 0; g4 < C / 4; ++g4) {
+        const float4 u = urow[g4];
+        w[4 * g4 + 0] = fmaf(-err, u.x, w[4 * g4 + 0]);
+        w[4 * g4 + 1] = fmaf(-err, u.y, w[4 * g4 + 1]);
+        w[4 * g4 + 2] = fmaf(-err, u.z, w[4 * g4 + 2]);
+        w[4 * g4 + 3] = fmaf(-err, u.w, w[4 * g4 + 3]);
       }
     }
   }
-  if (valid && a.row_loss != nullptr) a.row_loss[r] += loss;
+  if (!valid) return;
+  float* ehi = a.E_hi + r * a.lde + a.e_off;
+  float* elo = a.E_lo + r * a.lde + a.e_off;
+  uint8_t* crow = a.codes + r * a.n + a.i1;
+#pragma unroll
+  for (int m = 0; m < C; ++m) {
+    const int c = li + kLanes * m;
+    if (c < bw) {
+      const float h = __uint_as_float(__float_as_uint(e_own[m]) & 0xffffe000u);
+      ehi[c] = h;
+      elo[c] = e_own[m] - h;
+      crow[c] = static_cast<uint8_t>(q_own[m]);
+    }
+  }
+  if (li == 0 && a.row_loss != nullptr) a.row_loss[r] += loss;
 }
 
 // Per row, (min, max) of Wk[r, c0 : c1): the part of a group that lies past
@@ -383,21 +302,32 @@ __global__ void rtn_kernel(const T* __restrict__ W, int64_t rows, int n, int G, 
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Two-level lazy blocking: inside a super-block of about kSuper columns each
+// block's errors update only the super-block's remaining columns; the rest of
+// the matrix gets one update per super-block with K = the super-block width.
+// The same sums in another order (every column still receives every earlier
+// column's correction before it is quantized), so the outer updates are
+// GEMMs of K ~ 1024 instead of a read-modify-write of W per 128 columns.
+constexpr int kSuper = 1024;
+constexpr int kSuperMinN = 2 * kSuper;  // below this, one level
+
 struct QuantLayout {
   size_t wk, e_hi, e_lo, codes_p, u_hi, u_lo, minmax, total;
   int64_t ldu;
+  int lde;  // row pitch of the error buffers: one super-block (or one block)
 };
 
 QuantLayout quant_layout(int64_t rows, int n) {
   QuantLayout l{};
   l.ldu = (n + 3) / 4 * 4;  // 16-byte row pitch for the tensor-map loads
+  l.lde = n >= kSuperMinN ? kSuper : kBMax;
   size_t off = 0;
   l.wk = off;
   off += align256(static_cast<size_t>(rows) * n * sizeof(float));
   l.e_hi = off;
-  off += align256(static_cast<size_t>(rows) * kBMax * sizeof(float));
+  off += align256(static_cast<size_t>(rows) * l.lde * sizeof(float));
   l.e_lo = off;
-  off += align256(static_cast<size_t>(rows) * kBMax * sizeof(float));
+  off += align256(static_cast<size_t>(rows) * l.lde * sizeof(float));
   l.codes_p = off;
   off += align256(static_cast<size_t>(rows) * n);
   l.u_hi = off;
@@ -408,6 +338,15 @@ QuantLayout quant_layout(int64_t rows, int n) {
   off += align256(static_cast<size_t>(rows) * sizeof(float2));
   l.total = off;
   return l;
+}
+
+// Super-block width: a multiple of the block that fits the error buffers, and
+// one level when a group could reach past a super-block (its parameters are
+// fixed at its first column from fully updated weights).
+int super_width(const QuantLayout& l, int n, int block, int G) {
+  if (l.lde < kSuper) return block;
+  const int S = block * (kSuper / block);
+  return (G == n || S % G == 0) ? S : block;
 }
 
 }  // namespace
@@ -459,55 +398,53 @@ gptq_status quantize_layer(const void* W, gptq_dtype wdt, int64_t rows, int n, c
   a.maxq = static_cast<float>((1 << bits) - 1);
   a.E_hi = E_hi;
   a.E_lo = E_lo;
+  a.lde = l.lde;
   a.codes = codes_p;
   a.scales = scales;
   a.zeros = zeros;
   a.row_loss = row_loss;
-  a.block = block;
-  a.wait_ns = wait_limit_ns();
-  a.status = info->status;
-  // the U tile of each block arrives as one TMA box when U's rows are
-  // 16-byte aligned
-  CUtensorMap u_map;
-  std::memset(&u_map, 0, sizeof(u_map));
-  a.u_tma = (n % 4 == 0) ? 1 : 0;
-  if (a.u_tma && !make_tensor_map_2d(&u_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, U, static_cast<uint64_t>(n),
-                                     static_cast<uint64_t>(n), static_cast<uint64_t>(n) * 4, block, block,
-                                     CU_TENSOR_MAP_SWIZZLE_NONE))
-    return GPTQ_ERR_CUDA;
-  CUtensorMap uth_map, utl_map;
-  if (!make_tensor_map_2d(&uth_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, U_hi, static_cast<uint64_t>(n),
-                          static_cast<uint64_t>(n), static_cast<uint64_t>(l.ldu) * 4, block, block,
-                          CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_tensor_map_2d(&utl_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, U_lo, static_cast<uint64_t>(n),
-                          static_cast<uint64_t>(n), static_cast<uint64_t>(l.ldu) * 4, block, block,
-                          CU_TENSOR_MAP_SWIZZLE_NONE))
-    return GPTQ_ERR_CUDA;
-  const unsigned block_ctas = static_cast<unsigned>(ceil_div(rows, kRowsPerCta));
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(gptq_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kBlockSmem)) != cudaSuccess)
+  // kBlockLanes lanes per row; CTAs of up to 32 warps, sized so that two
+  // CTAs per SM cover the rows in one wave
+  constexpr int rows_per_warp = 32 / kBlockLanes;
+  const size_t block_smem = BlockShape<kBlockLanes>::kSmem;
+  const int64_t warps_needed = ceil_div(rows, static_cast<int64_t>(rows_per_warp));
+  const int64_t want = ceil_div(warps_needed, static_cast<int64_t>(2 * info->sm_count));
+  const int warps_per_cta = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(kMaxWarpsPerCta, want)));
+  const unsigned block_ctas = static_cast<unsigned>(ceil_div(warps_needed, static_cast<int64_t>(warps_per_cta)));
+  static bool attr_set[64] = {};
+  if (!attr_set[info->device]) {
+    if (cudaFuncSetAttribute(gptq_block_kernel<kBlockLanes>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(block_smem)) != cudaSuccess)
       return GPTQ_ERR_CUDA;
-    attr_set = true;
+    attr_set[info->device] = true;
   }
-  for (int i1 = 0; i1 < n; i1 += block) {
-    a.i1 = i1;
-    a.bw = std::min(block, n - i1);
-    // a group that starts here and runs past the block: min / max of its
-    // columns beyond the block, taken before the block changes anything
-    const int gend = std::min(i1 + G, n);
-    a.ext_minmax = nullptr;
-    if (i1 % G == 0 && i1 + a.bw < gend) {
-      launch(group_minmax_kernel, static_cast<unsigned>(ceil_div(rows * 32, 256)), 256, 0, st, Wk, rows, n,
-             i1 + a.bw, gend, ext_minmax);
-      a.ext_minmax = ext_minmax;
+  const int S = super_width(l, n, block, G);
+  for (int s1 = 0; s1 < n; s1 += S) {
+    const int s2 = std::min(s1 + S, n);
+    for (int i1 = s1; i1 < s2; i1 += block) {
+      a.i1 = i1;
+      a.bw = std::min(block, s2 - i1);
+      a.e_off = i1 - s1;
+      // a group that starts here and runs past the block: min / max of its
+      // columns beyond the block, taken before the block changes anything
+      const int gend = std::min(i1 + G, n);
+      a.ext_minmax = nullptr;
+      if (i1 % G == 0 && i1 + a.bw < gend) {
+        launch(group_minmax_kernel, static_cast<unsigned>(ceil_div(rows * 32, 256)), 256, 0, st, Wk, rows, n,
+               i1 + a.bw, gend, ext_minmax);
+        a.ext_minmax = ext_minmax;
+      }
+      launch(gptq_block_kernel<kBlockLanes>, block_ctas, warps_per_cta * 32, block_smem, st, a);
+      const int i2 = i1 + a.bw;
+      if (i2 < s2) {  // inner update: the rest of the super-block
+        const gptq_status ts = trailing_update_tc(Wk, n, static_cast<int>(rows), s2 - i2, a.bw, i2, i1, E_hi + a.e_off,
+                                                  E_lo + a.e_off, l.lde, U_hi, U_lo, l.ldu, n, st);
+        if (ts != GPTQ_OK) return ts;
+      }
     }
-    launch(gptq_block_kernel, block_ctas, kRowsPerCta, kBlockSmem, st, u_map, uth_map, utl_map, a);
-    const int i2 = i1 + a.bw;
-    if (i2 < n) {
-      const gptq_status ts = trailing_update_tc(Wk, n, static_cast<int>(rows), n - i2, a.bw, i2, i1, E_hi, E_lo,
-                                                kBMax, U_hi, U_lo, l.ldu, n, st);
+    if (s2 < n) {  // outer update: everything after the super-block
+      const gptq_status ts = trailing_update_tc(Wk, n, static_cast<int>(rows), n - s2, s2 - s1, s2, s1, E_hi, E_lo,
+                                                l.lde, U_hi, U_lo, l.ldu, n, st);
       if (ts != GPTQ_OK) return ts;
     }
   }

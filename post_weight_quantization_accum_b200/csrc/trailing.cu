@@ -295,9 +295,10 @@ gptq_status trailing_update_tc(float* W, int64_t ldw, int M, int N, int K, int c
   if (K % kBK != 0) return GPTQ_ERR_INVALID_ARG;
   CUtensorMap m_ehi, m_elo, m_uhi, m_ulo;
   const CUtensorMapDataType f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-  if (!make_tensor_map_2d(&m_ehi, f32, E_hi, static_cast<uint64_t>(lde), static_cast<uint64_t>(M),
+  // E's maps span exactly the K columns used (the base may sit inside a row)
+  if (!make_tensor_map_2d(&m_ehi, f32, E_hi, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
                           static_cast<uint64_t>(lde) * 4, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tensor_map_2d(&m_elo, f32, E_lo, static_cast<uint64_t>(lde), static_cast<uint64_t>(M),
+      !make_tensor_map_2d(&m_elo, f32, E_lo, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
                           static_cast<uint64_t>(lde) * 4, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tensor_map_2d(&m_uhi, f32, U_hi, static_cast<uint64_t>(n_u), static_cast<uint64_t>(n_u),
                           static_cast<uint64_t>(ldu) * 4, kBK, kBN, CU_TENSOR_MAP_SWIZZLE_128B) ||

@@ -66,6 +66,34 @@ def test_column_loop_with_identity_factor_is_rtn(bits, group, block):
     assert np.array_equal(npx(out["deq"]), ref["deq"])
 
 
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_column_loop_codes_at_grid_decision_points(bits):
+    """Weights within a few ulps of the grid's half-way points between codes
+    (where w / scale rounds either way): with U = I the column loop is RTN, and
+    its codes, scales and dequantized values equal the float32 oracle's exactly."""
+    maxq = (1 << bits) - 1
+    rows, n, G = 48, 512, 128
+    rng = np.random.default_rng(100 + bits)
+    W = np.zeros((rows, n), np.float32)
+    for r in range(rows):
+        for g0 in range(0, n, G):
+            a, b = np.float32(rng.uniform(0.01, 0.05)), np.float32(rng.uniform(0.01, 0.05))
+            scale, zero = go.group_params_f32(np.array([[-a, b]], np.float32), maxq)
+            s, z = np.float32(scale[0]), int(zero[0])
+            k = rng.integers(-z, maxq - z, size=G - 2)
+            vals = ((k + 0.5).astype(np.float32) * s).astype(np.float32)
+            for i, st in enumerate(rng.integers(-3, 4, size=G - 2)):
+                for _ in range(abs(int(st))):
+                    vals[i] = np.nextafter(vals[i], np.float32(np.inf if st > 0 else -np.inf))
+            W[r, g0:g0 + G] = np.concatenate([[-a, b], np.clip(vals, -a, b)]).astype(np.float32)
+    Wt = torch.tensor(W, device="cuda")
+    out = gq.gptq_quantize_layer(Wt, torch.eye(n, device="cuda"), bits, G, 128, want_deq=True)
+    ref = go.rtn_quantize_f32(W, bits, G)
+    assert np.array_equal(npx(out["codes"]).astype(np.int64), ref["codes"])
+    assert np.array_equal(npx(out["scales"]), ref["scales"].astype(np.float32))
+    assert np.array_equal(npx(out["deq"]), ref["deq"])
+
+
 # ---------------------------------------------------------------------------
 # packing: bit-exact
 # ---------------------------------------------------------------------------
@@ -227,6 +255,22 @@ def test_block_size_invariance_on_gpu(block, group):
     out, ref, agree, err_gpu, err_ref = _layer_parity(spec)
     assert agree >= 0.999
     assert abs(err_gpu - err_ref) <= 1e-3 * err_ref
+
+
+@pytest.mark.parametrize("name,rows,n,group,block", [
+    ("attn4096", 48, 2048, 128, 128),   # two super-blocks of 1024 columns
+    ("layer256", 32, 2048, 0, 96),      # per-row grid, super-blocks of 960: 960, 960 and a ragged 128
+    ("mlp_up", 32, 2304, 128, 128),     # act-order, 3-bit: 1024, 1024, 256
+    ("attn4096", 32, 2304, 384, 128),   # groups of 384 do not divide 1024: one level
+])
+def test_two_level_blocking_matches_oracle(name, rows, n, group, block):
+    """Layers wide enough for super-blocks (inner updates inside 1024 columns,
+    one outer update per super-block) against the oracle's plain block loop."""
+    spec = si.scaled(si.SPECS[name], rows=rows, n=n, n_tok=4096, group=group, block=block)
+    out, ref, agree, err_gpu, err_ref = _layer_parity(spec)
+    assert agree >= 0.999, agree
+    assert abs(err_gpu - err_ref) <= 1e-3 * err_ref, (err_gpu, err_ref)
+    np.testing.assert_allclose(npx(out["row_loss"]), ref["row_loss"], rtol=2e-2)
 
 
 def test_dead_columns_and_bf16_weights():
