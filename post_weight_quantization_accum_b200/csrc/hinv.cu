@@ -133,6 +133,7 @@ struct CholArgs {
   unsigned* bar;     // grid barrier: [0] arrivals, [1] generation (zeroed on entry)
   int* abort;        // set when a barrier wait runs out (zeroed on entry)
   uint64_t wait_ns;
+  int vec;           // n % 4 == 0: rows of four along a tile row are 16-byte aligned
 };
 
 typedef float Tile[kPad];
@@ -147,9 +148,6 @@ __device__ __forceinline__ float* at_a(const CholArgs& p, int r, int c) { return
 __device__ __forceinline__ float* at_x(const CholArgs& p, int r, int c) {
   return p.U + static_cast<size_t>(p.n - 1 - r) * p.n + (p.n - 1 - c);
 }
-
-// A thread holds 16 elements of each 64 x 64 tile it stages.
-constexpr int kPerThread = kT * kT / kCholThreads;  // 16
 
 // acc[i][j] = sum_k P[k][tr+i] * Q[k][tc+j]  (thread owns a 4x4 block)
 __device__ __forceinline__ void tile_product(const Tile* P, const Tile* Q, float (&acc)[4][4]) {
@@ -323,33 +321,99 @@ __device__ __forceinline__ TileOp op_phase_u(int k, int nb, int t) {
   return {kOpInverse, (k + 1 + tt / (k + 1)) * kT, (tt % (k + 1)) * kT};
 }
 
+// Four consecutive entries (r, c .. c + 3) of A or of X (X rotated into U,
+// so they lie in reverse order); c % 4 == 0.  Vector loads when p.vec.
+__device__ __forceinline__ float4 ld4_a(const CholArgs& p, int r, int c) {
+  if (r >= p.n || c >= p.n) return make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  const float* src = p.A + static_cast<size_t>(r) * p.n + c;
+  if (p.vec) return __ldcg(reinterpret_cast<const float4*>(src));
+  return make_float4(__ldcg(src), c + 1 < p.n ? __ldcg(src + 1) : 0.0f, c + 2 < p.n ? __ldcg(src + 2) : 0.0f,
+                     c + 3 < p.n ? __ldcg(src + 3) : 0.0f);
+}
+__device__ __forceinline__ float4 ld4_x(const CholArgs& p, int r, int c) {
+  if (r >= p.n || c >= p.n) return make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  const float* row = p.U + static_cast<size_t>(p.n - 1 - r) * p.n + (p.n - 1);
+  if (p.vec) {
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(row - c - 3));
+    return make_float4(v.w, v.z, v.y, v.x);
+  }
+  return make_float4(__ldcg(row - c), c + 1 < p.n ? __ldcg(row - c - 1) : 0.0f,
+                     c + 2 < p.n ? __ldcg(row - c - 2) : 0.0f, c + 3 < p.n ? __ldcg(row - c - 3) : 0.0f);
+}
+__device__ __forceinline__ void st4(const CholArgs& p, bool to_x, int r, int c, float4 v) {
+  if (r >= p.n || c >= p.n) return;
+  if (!to_x) {
+    float* dst = p.A + static_cast<size_t>(r) * p.n + c;
+    if (p.vec) {
+      *reinterpret_cast<float4*>(dst) = v;
+    } else {
+      dst[0] = v.x;
+      if (c + 1 < p.n) dst[1] = v.y;
+      if (c + 2 < p.n) dst[2] = v.z;
+      if (c + 3 < p.n) dst[3] = v.w;
+    }
+  } else {
+    float* row = p.U + static_cast<size_t>(p.n - 1 - r) * p.n + (p.n - 1);
+    if (p.vec) {
+      *reinterpret_cast<float4*>(row - c - 3) = make_float4(v.w, v.z, v.y, v.x);
+    } else {
+      row[-c] = v.x;
+      if (c + 1 < p.n) row[-c - 1] = v.y;
+      if (c + 2 < p.n) row[-c - 2] = v.z;
+      if (c + 3 < p.n) row[-c - 3] = v.w;
+    }
+  }
+}
+
+// Which four entries (row a, columns 4 b4 .. 4 b4 + 3) of a 64 x 64 operand
+// thread t stages in its slot g.  An operand that shared memory keeps
+// transposed uses mapping T: two lanes per row (one 32-byte sector per row and
+// instruction), so that the transposed scalar stores of a warp hit 32
+// distinct banks.  One kept as loaded uses mapping N: 16 lanes along a row,
+// conflict-free vector stores.
+__device__ __forceinline__ void slot_t(int g, int& a, int& b4) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  a = (lane >> 1) + 16 * (warp & 3);
+  b4 = (lane & 1) + 2 * ((warp >> 2) + 2 * g);
+}
+__device__ __forceinline__ void slot_n(int g, int& a, int& b4) {
+  const int idx = g * kCholThreads + threadIdx.x;
+  a = idx >> 4;
+  b4 = idx & 15;
+}
+
 // Registers holding one tile operation's operands (and, for the subtracting
 // operations, the old output values) between its loads and its use.
 struct Staged {
-  float p[kPerThread], q[kPerThread], o[kPerThread];
+  float4 p[4], q[4], o[4];
 };
+
+__device__ __forceinline__ bool q_natural(const TileOp& op) { return op.kind == kOpFinalize || op.kind == kOpInverse; }
 
 __device__ __forceinline__ void fetch_op(const CholArgs& p, const TileOp& op, int k0, Staged& st) {
   const int tr = (threadIdx.x / 16) * 4, tc = (threadIdx.x % 16) * 4;
 #pragma unroll
-  for (int q = 0; q < kPerThread; ++q) {
-    const int e = threadIdx.x + q * kCholThreads, a = e / kT, b = e % kT;
+  for (int g = 0; g < 4; ++g) {
+    int a, b4, an, bn4;
+    slot_t(g, a, b4);
+    slot_n(g, an, bn4);
+    const int b = 4 * b4;
     switch (op.kind) {
       case kOpTrsm:      // A_ik * Linv_kk^T
-        st.p[q] = ld_a(p, op.i0 + a, k0 + b);
-        st.q[q] = ld_x(p, k0 + a, k0 + b);
+        st.p[g] = ld4_a(p, op.i0 + a, k0 + b);
+        st.q[g] = ld4_x(p, k0 + a, k0 + b);
         break;
       case kOpFinalize:  // Linv_kk * R_kj
-        st.p[q] = ld_x(p, k0 + a, k0 + b);
-        st.q[q] = ld_x(p, k0 + a, op.j0 + b);
+        st.p[g] = ld4_x(p, k0 + a, k0 + b);
+        st.q[g] = ld4_x(p, k0 + an, op.j0 + 4 * bn4);
         break;
       case kOpUpdate:    // A_ij - L_ik L_jk^T
-        st.p[q] = ld_a(p, op.i0 + a, k0 + b);
-        st.q[q] = ld_a(p, op.j0 + a, k0 + b);
+        st.p[g] = ld4_a(p, op.i0 + a, k0 + b);
+        st.q[g] = ld4_a(p, op.j0 + a, k0 + b);
         break;
       default:           // R_ij - L_ik X_kj
-        st.p[q] = ld_a(p, op.i0 + a, k0 + b);
-        st.q[q] = ld_x(p, k0 + a, op.j0 + b);
+        st.p[g] = ld4_a(p, op.i0 + a, k0 + b);
+        st.q[g] = ld4_x(p, k0 + an, op.j0 + 4 * bn4);
         break;
     }
   }
@@ -357,29 +421,38 @@ __device__ __forceinline__ void fetch_op(const CholArgs& p, const TileOp& op, in
     const bool to_x = op.kind == kOpInverse;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        st.o[4 * i + j] = to_x ? ld_x(p, op.i0 + tr + i, op.j0 + tc + j) : ld_a(p, op.i0 + tr + i, op.j0 + tc + j);
+      st.o[i] = to_x ? ld4_x(p, op.i0 + tr + i, op.j0 + tc) : ld4_a(p, op.i0 + tr + i, op.j0 + tc);
   }
 }
 
 // P is always used as P[r][k]; Q as Q[c][k] (transposed load) for the
 // Cholesky operations and as Q[k][c] (natural load) for the inverse ones.
 __device__ __forceinline__ void commit_op(const TileOp& op, const Staged& st, Tile* sp, Tile* sq) {
-  const bool q_natural = op.kind == kOpFinalize || op.kind == kOpInverse;
+  const bool qn = q_natural(op);
 #pragma unroll
-  for (int q = 0; q < kPerThread; ++q) {
-    const int e = threadIdx.x + q * kCholThreads, a = e / kT, b = e % kT;
-    sp[b][a] = st.p[q];
-    if (q_natural)
-      sq[a][b] = st.q[q];
-    else
-      sq[b][a] = st.q[q];
+  for (int g = 0; g < 4; ++g) {
+    int a, b4;
+    slot_t(g, a, b4);
+    const int b = 4 * b4;
+    sp[b + 0][a] = st.p[g].x;
+    sp[b + 1][a] = st.p[g].y;
+    sp[b + 2][a] = st.p[g].z;
+    sp[b + 3][a] = st.p[g].w;
+    if (qn) {
+      int an, bn4;
+      slot_n(g, an, bn4);
+      *reinterpret_cast<float4*>(&sq[an][4 * bn4]) = st.q[g];
+    } else {
+      sq[b + 0][a] = st.q[g].x;
+      sq[b + 1][a] = st.q[g].y;
+      sq[b + 2][a] = st.q[g].z;
+      sq[b + 3][a] = st.q[g].w;
+    }
   }
 }
 
 __device__ __forceinline__ void finish_op(const CholArgs& p, const TileOp& op, int k0, const float (&acc)[4][4],
-                                          const float* old) {
+                                          const float4* old) {
   const int tr = (threadIdx.x / 16) * 4, tc = (threadIdx.x % 16) * 4;
   const bool to_x = op.kind == kOpFinalize || op.kind == kOpInverse;
   const bool subtract = op.kind == kOpUpdate || op.kind == kOpInverse;
@@ -387,15 +460,12 @@ __device__ __forceinline__ void finish_op(const CholArgs& p, const TileOp& op, i
   const int c0 = op.kind == kOpTrsm ? k0 : op.j0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int r = r0 + tr + i;
-    if (r >= p.n) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int c = c0 + tc + j;
-      if (c >= p.n) continue;
-      float* dst = to_x ? at_x(p, r, c) : at_a(p, r, c);
-      *dst = subtract ? old[4 * i + j] - acc[i][j] : acc[i][j];
+    float4 v = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+    if (subtract) {
+      const float4 o = old[i * kCholThreads];
+      v = make_float4(o.x - v.x, o.y - v.y, o.z - v.z, o.w - v.w);
     }
+    st4(p, to_x, r0 + tr + i, c0 + tc, v);
   }
 }
 
@@ -411,10 +481,10 @@ __device__ void run_phase(const CholArgs& p, int k, int t0, int step, int total,
   fetch_op(p, cur, k0, st);
   for (int t = t0; t < total; t += step) {
     commit_op(cur, st, s0, s1);
-    // the old output values wait in this thread's own slots of s2
-    float* old = &s2[0][0] + threadIdx.x * kPerThread;
+    // the old output values wait in s2 (float4 slot [i][thread], conflict-free)
+    float4* old = reinterpret_cast<float4*>(&s2[0][0]) + threadIdx.x;
 #pragma unroll
-    for (int q = 0; q < kPerThread; ++q) old[q] = st.o[q];
+    for (int i = 0; i < 4; ++i) old[i * kCholThreads] = st.o[i];
     __syncthreads();
     const int tn = t + step;
     TileOp nxt = cur;
@@ -550,6 +620,7 @@ gptq_status prepare_hinv(const float* H, const double* hdiag, int n, float damp,
   ca.bar = bar;
   ca.abort = reinterpret_cast<int*>(bar + 2);
   ca.wait_ns = wait_limit_ns();
+  ca.vec = (n % 4 == 0) ? 1 : 0;
   void* args[] = {&ca};
   if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(chol_inv_kernel), dim3(grid), dim3(kCholThreads),
                                   args, kCholSmem, st) != cudaSuccess)
