@@ -5,25 +5,34 @@
 // token-major (X[t, i], bf16), so the product is X^T X: a symmetric rank-N
 // update (SYRK) whose inner dimension is the token count.
 //
-// Kernel design (one CTA per SM, persistent):
-//   * Output tiles of 128 rows x 256 columns cover the lower triangle in
-//     128-row blocks; the last tile of an even row block is 128 wide.
+// Kernel design (persistent CTA pairs, one CTA per SM):
+//   * Output tiles of 256 x 256 cover the lower triangle in 256-row blocks.
+//     A cluster of two CTAs (one TPC) computes a tile with tcgen05 pair MMAs
+//     (cta_group::2, M = 256, N = 256, K = 16): each CTA loads half of the
+//     rows' features (A, 128) and half of the columns' features (B, 128) and
+//     holds its 128 rows of the fp32 accumulator in its own tensor memory.
+//     Per CTA and stage that is 32 KB of operands for 2 * 128 * 256 * 64
+//     flops, a third less shared-memory and L2 traffic per flop than a
+//     single-CTA 128 x 256 tile.
 //   * Both operands are slices of the same X tile stream and are MN-major
 //     (features contiguous): TMA loads 64-feature x 64-token boxes with the
-//     128-byte swizzle into a 4-stage shared-memory ring.
-//   * One thread issues tcgen05.mma (kind::f16, bf16 x bf16 -> fp32, M=128,
-//     N=256|128, K=16) into a double-buffered tensor-memory accumulator
-//     (2 x 256 columns), so the epilogue of one work unit overlaps the next.
+//     128-byte swizzle into a 6-stage ring; both CTAs' loads are counted on
+//     the even CTA's barrier, whose single thread issues the MMAs; MMA
+//     completion is signalled to both CTAs (commit multicast), which frees
+//     their stages and hands the accumulators to their epilogue warps.
+//   * The accumulator is double-buffered (2 x 256 columns), so the epilogue
+//     of one work unit overlaps the next.
 //   * The token range is cut into `splits` equal chunks; work unit u covers
-//     tile (u % tiles) over chunk (u / tiles) and CTAs take units round-robin.
-//     All CTAs therefore sweep the tokens in the same order, which keeps the
-//     X slice they share resident in L2.  Each unit writes its fp32 partial
-//     tile to the workspace; a finalize kernel sums the partials in a fixed
-//     order, scales by alpha and adds into both triangles of H, so the result
-//     is deterministic and exactly symmetric.
+//     tile (u % tiles) over chunk (u / tiles) and pairs take units
+//     round-robin, so all pairs sweep the tokens in the same order and the
+//     X slice they share stays in L2.  Each unit writes its fp32 partial tile
+//     to the workspace; a finalize kernel sums the partials in a fixed order,
+//     scales by alpha and adds into both triangles of H, so the result is
+//     deterministic and exactly symmetric.
 //   * Every barrier wait is bounded in time; a wait that runs out records
-//     GPTQ_ERR_TIMEOUT, stops the CTA's loops, waits (bounded) for its own
-//     in-flight copies and MMAs and releases tensor memory before returning.
+//     GPTQ_ERR_TIMEOUT and stops the CTA's loops; the CTA then waits (bounded)
+//     for the copies and MMAs it is responsible for, meets its peer at a
+//     cluster barrier and releases tensor memory before returning.
 //
 // The fp64 diagonal (act-order key) is accumulated by a separate pair of
 // kernels with a fixed summation order.
@@ -36,16 +45,15 @@
 namespace gptq {
 namespace {
 
-constexpr int kBM = 128;                          // tile rows
-constexpr int kBNMax = 256;                       // tile columns
+constexpr int kTile = 256;                        // output tile rows = columns (one CTA pair)
+constexpr int kHalf = 128;                        // features per CTA for each operand
 constexpr int kBK = 64;                           // tokens per pipeline stage
-constexpr int kStages = 4;
+constexpr int kStages = 6;
 constexpr int kBoxBytes = 64 * kBK * 2;           // one 64-feature x 64-token bf16 box
-constexpr int kABytes = kBM * kBK * 2;            // 16 KB
-constexpr int kBBytes = kBNMax * kBK * 2;         // 32 KB
-constexpr int kStageBytes = kABytes + kBBytes;    // 48 KB
+constexpr int kHalfBytes = kHalf * kBK * 2;       // 16 KB: one operand half
+constexpr int kStageBytes = 2 * kHalfBytes;       // A half + B half = 32 KB per CTA
 constexpr int kThreads = 192;                     // producer, MMA, 4 epilogue warps
-constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemCols = 512;               // 2 x 256-column accumulators
 constexpr int kBarrierBytes = 256;
 constexpr size_t kSmemBytes = 1024 + size_t(kStages) * kStageBytes + kBarrierBytes;
 constexpr uint64_t kDrainNs = 2000000000ull;      // bound for draining in-flight work
@@ -60,29 +68,18 @@ struct SyrkParams {
   uint64_t wait_ns;
 };
 
-// Tile t -> (row block, first column, width).  Row block rb holds
-// ceil((rb + 1) / 2) tiles; m(m+1) tiles precede row block 2m and (m+1)^2
-// precede row block 2m+1.
-__host__ __device__ inline void tile_coords(int t, int& rb, int& c0, int& N) {
-  int m = static_cast<int>((sqrtf(4.0f * static_cast<float>(t) + 1.0f) - 1.0f) * 0.5f);
-  while ((m + 1) * (m + 2) <= t) ++m;
-  while (m > 0 && m * (m + 1) > t) --m;
-  int idx;
-  if (t < (m + 1) * (m + 1)) {
-    rb = 2 * m;
-    idx = t - m * (m + 1);
-  } else {
-    rb = 2 * m + 1;
-    idx = t - (m + 1) * (m + 1);
-  }
-  c0 = idx * kBNMax;
-  N = min(kBNMax, (rb + 1) * kBM - c0);
+// Tile t -> (row block, column block) with t = rb (rb + 1) / 2 + cb, cb <= rb.
+__host__ __device__ inline void tile_coords(int t, int& rb, int& cb) {
+  int r = static_cast<int>((sqrtf(8.0f * static_cast<float>(t) + 1.0f) - 1.0f) * 0.5f);
+  while ((r + 1) * (r + 2) / 2 <= t) ++r;
+  while (r > 0 && r * (r + 1) / 2 > t) --r;
+  rb = r;
+  cb = t - r * (r + 1) / 2;
 }
 
 inline int tiles_for(int n) {
-  const int rb = static_cast<int>(ceil_div(n, kBM));
-  const int m = rb / 2;
-  return (rb % 2 == 0) ? m * (m + 1) : (m + 1) * (m + 1);
+  const int rbs = static_cast<int>(ceil_div(n, kTile));
+  return rbs * (rbs + 1) / 2;
 }
 
 __device__ __forceinline__ void unit_range(const SyrkParams& p, int u, int& t, int& kb0, int& kb1) {
@@ -107,15 +104,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_ctarank();  // 0: issues the MMAs; 1: its peer
+  const int pair = static_cast<int>(blockIdx.x) / 2;
+  const int pairs = static_cast<int>(gridDim.x) / 2;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(full + s, 1);
-      mbar_init(empty + s, 1);
+      mbar_init(full + s, 1);   // the even CTA's expect-tx arrival (+ both CTAs' bytes)
+      mbar_init(empty + s, 1);  // one MMA commit per stage use
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(acc_full + b, 1);
-      mbar_init(acc_empty + b, 4);
+      mbar_init(acc_full + b, 1);   // one MMA commit per work unit
+      mbar_init(acc_empty + b, 8);  // four epilogue warps of each CTA
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -123,26 +123,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&xmap);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // barriers of both CTAs initialised before any cross-CTA use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int num_units = p.splits * p.tiles;
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producer ----------------
+      // ---------------- TMA producer (both CTAs) ----------------
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued = 0, issued_parity = 0;  // per-stage bits for the drain
-      for (int u = blockIdx.x; u < num_units && !*abort_flag; u += gridDim.x) {
-        int t, kb0, kb1, rb, c0, N;
+      for (int u = pair; u < num_units && !*abort_flag; u += pairs) {
+        int t, kb0, kb1, rb, cb;
         unit_range(p, u, t, kb0, kb1);
-        tile_coords(t, rb, c0, N);
-        const uint32_t bytes = static_cast<uint32_t>((kBM + N) * kBK * 2);
+        tile_coords(t, rb, cb);
+        const int fa = rb * kTile + static_cast<int>(rank) * kHalf;  // this CTA's A features
+        const int fb = cb * kTile + static_cast<int>(rank) * kHalf;  // this CTA's B features
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(empty + stage, phase ^ 1u, p.wait_ns)) {
             set_status(p.status, GPTQ_ERR_TIMEOUT);
@@ -151,12 +153,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (*abort_flag) break;
           uint8_t* a = ring + size_t(stage) * kStageBytes;
-          uint8_t* b = a + kABytes;
+          uint8_t* b = a + kHalfBytes;
           const int y = kb * kBK;
-          mbar_arrive_expect_tx(full + stage, bytes);
-          tma_load_2d(a, &xmap, full + stage, rb * kBM, y);
-          tma_load_2d(a + kBoxBytes, &xmap, full + stage, rb * kBM + 64, y);
-          for (int j = 0; j < N / 64; ++j) tma_load_2d(b + j * kBoxBytes, &xmap, full + stage, c0 + 64 * j, y);
+          const uint32_t bar = smem_cluster_addr(full + stage, 0);
+          if (rank == 0) mbar_arrive_expect_tx(full + stage, 2u * kStageBytes);
+          tma_load_2d_pair(a, &xmap, bar, fa, y);
+          tma_load_2d_pair(a + kBoxBytes, &xmap, bar, fa + 64, y);
+          tma_load_2d_pair(b, &xmap, bar, fb, y);
+          tma_load_2d_pair(b + kBoxBytes, &xmap, bar, fb + 64, y);
           issued |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == kStages) {
@@ -165,25 +169,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      // Drain: every box this thread issued has landed before the CTA exits.
-      for (int s = 0; s < kStages; ++s) {
-        if (issued & (1u << s)) {
-          if (!mbar_wait(full + s, (issued_parity >> s) & 1u, kDrainNs)) set_status(p.status, GPTQ_ERR_TIMEOUT);
+      // Drain (even CTA): every stage it armed has received both CTAs' bytes.
+      if (rank == 0) {
+        for (int s = 0; s < kStages; ++s) {
+          if (issued & (1u << s)) {
+            if (!mbar_wait(full + s, (issued_parity >> s) & 1u, kDrainNs)) set_status(p.status, GPTQ_ERR_TIMEOUT);
+          }
         }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer ----------------
+    if (lane == 0 && rank == 0) {
+      // ---------------- MMA issuer (even CTA) ----------------
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x, ++local) {
-        int t, kb0, kb1, rb, c0, N;
+      const uint32_t idesc = instr_desc(1u, 1u, 1u, kTile, kTile);
+      for (int u = pair; u < num_units && ok; u += pairs, ++local) {
+        int t, kb0, kb1;
         unit_range(p, u, t, kb0, kb1);
-        tile_coords(t, rb, c0, N);
-        const uint32_t idesc = instr_desc(1u, 1u, 1u, kBM, static_cast<uint32_t>(N));
         const int buf = local & 1;
         const uint32_t acc_phase = static_cast<uint32_t>(local >> 1) & 1u;
         if (!mbar_wait(acc_empty + buf, acc_phase ^ 1u, p.wait_ns) || *abort_flag) {
@@ -192,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kBNMax);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kTile);
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(full + stage, phase, p.wait_ns) || *abort_flag) {
             set_status(p.status, GPTQ_ERR_TIMEOUT);
@@ -202,35 +207,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(ring + size_t(stage) * kStageBytes);
-          const uint32_t b_addr = a_addr + kABytes;
+          const uint32_t b_addr = a_addr + kHalfBytes;
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
             const uint64_t adesc = smem_desc_sw128(a_addr + kk * 2048, kBoxBytes, 1024);
             const uint64_t bdesc = smem_desc_sw128(b_addr + kk * 2048, kBoxBytes, 1024);
-            mma_f16(d_tmem, adesc, bdesc, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+            mma_f16_pair(d_tmem, adesc, bdesc, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(empty + stage);
+          mma_commit_pair(empty + stage, 0x3);
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        mma_commit(acc_full + buf);
+        mma_commit_pair(acc_full + buf, 0x3);
       }
-      // Drain: all MMAs this thread issued have completed.
-      mma_commit(drain);
+      // Drain: all pair MMAs issued have completed (they read both CTAs' stages).
+      mma_commit_pair(drain, 0x1);
       if (!mbar_wait(drain, 0u, kDrainNs)) set_status(p.status, GPTQ_ERR_TIMEOUT);
     }
   } else {
-    // ---------------- epilogue: TMEM -> registers -> workspace ----------------
+    // ---------------- epilogue (both CTAs): TMEM -> registers -> workspace ----------------
     const int quad = warp & 3;  // tensor-memory lanes this warp may access
-    const int row = quad * 32 + lane;
+    const int row = static_cast<int>(rank) * kHalf + quad * 32 + lane;
     int local = 0;
-    for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++local) {
-      int t, kb0, kb1, rb, c0, N;
-      unit_range(p, u, t, kb0, kb1);
-      tile_coords(t, rb, c0, N);
+    for (int u = pair; u < num_units; u += pairs, ++local) {
       const int buf = local & 1;
       const uint32_t acc_phase = static_cast<uint32_t>(local >> 1) & 1u;
       // lane 0 waits and the warp follows its verdict, so the warp stays
@@ -246,10 +248,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      float* dst = p.partial + (static_cast<size_t>(u) * kBM + row) * kBNMax;
-      for (int c = 0; c < N; c += 32) {
+      float* dst = p.partial + (static_cast<size_t>(u) * kTile + row) * kTile;
+      for (int c = 0; c < kTile; c += 32) {
         uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(buf * kBNMax + c), r);
+        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(buf * kTile + c), r);
         tmem_ld_wait();
         float4* d4 = reinterpret_cast<float4*>(dst + c);
 #pragma unroll
@@ -259,38 +261,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty + buf);
+      if (lane == 0) mbar_arrive_cluster(smem_cluster_addr(acc_empty + buf, 0));
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // neither CTA leaves while the pair still uses its memory
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    tmem_dealloc_pair(tmem_base, kTmemCols);
   }
 }
 
 // Sums the partial tiles of every token chunk in chunk order, scales by alpha
 // and adds the lower triangle into H and its mirror image into the upper one.
-// Grid (tiles, 8, 4) x block (32, 8): one 32x32 sub-block per CTA.
+// Grid (tiles, 8, 8) x block (32, 8): one 32x32 sub-block per CTA.
 __global__ void syrk_finalize_kernel(const float* __restrict__ partial, float* __restrict__ H, int n, int tiles,
                                      int splits, float alpha) {
-  int rb, c0, N;
-  tile_coords(blockIdx.x, rb, c0, N);
+  int rb, cb;
+  tile_coords(blockIdx.x, rb, cb);
   const int sc = blockIdx.y * 32;
   const int sr = blockIdx.z * 32;
-  if (sc >= N) return;
-  const int r0 = rb * kBM + sr;
-  const int cc0 = c0 + sc;
+  const int r0 = rb * kTile + sr;
+  const int cc0 = cb * kTile + sc;
   if (r0 >= n || cc0 >= n || cc0 > r0 + 31) return;
   __shared__ float tr[32][33];
   const int tx = threadIdx.x;
   for (int i = threadIdx.y; i < 32; i += 8) {
     float v = 0.0f;
     for (int s = 0; s < splits; ++s)
-      v += partial[(static_cast<size_t>(s * tiles + blockIdx.x) * kBM + sr + i) * kBNMax + sc + tx];
+      v += partial[(static_cast<size_t>(s * tiles + blockIdx.x) * kTile + sr + i) * kTile + sc + tx];
     v *= alpha;
     tr[tx][i] = v;
     const int r = r0 + i, c = cc0 + tx;
@@ -333,26 +335,17 @@ __global__ void hdiag_reduce_kernel(const double* __restrict__ part, int chunks,
 }
 
 // Token chunks for the split-K schedule: the smallest count (<= 16) whose
-// round-robin assignment keeps the busiest CTA within 5% of the average,
-// else the best balance found.
-int choose_splits(int n, int64_t n_tok, int ctas) {
+// round-robin assignment of units to CTA pairs keeps the busiest pair within
+// 5% of the average, else the best balance found.  Tiles are equal in cost.
+int choose_splits(int n, int64_t n_tok, int pairs) {
   const int tiles = tiles_for(n);
   const int64_t kblocks = ceil_div(n_tok, kBK);
   double best_eff = -1.0;
   int best = 1;
   for (int s = 1; s <= 16 && s <= kblocks; ++s) {
     const int units = s * tiles;
-    const int grid = std::min(ctas, units);
-    std::vector<double> load(grid, 0.0);
-    double total = 0.0;
-    for (int u = 0; u < units; ++u) {
-      int rb, c0, N;
-      tile_coords(u % tiles, rb, c0, N);
-      const double w = static_cast<double>(kBM + N) * N;  // MMA plus operand-load cost
-      load[u % grid] += w;
-      total += w;
-    }
-    const double eff = total / (static_cast<double>(ctas) * *std::max_element(load.begin(), load.end()));
+    const int busiest = static_cast<int>(ceil_div(units, pairs));
+    const double eff = static_cast<double>(units) / (static_cast<double>(pairs) * busiest);
     if (eff >= 0.95) return s;
     if (eff > best_eff + 1e-9) {
       best_eff = eff;
@@ -362,8 +355,10 @@ int choose_splits(int n, int64_t n_tok, int ctas) {
   return best;
 }
 
+int pairs_for(const DeviceInfo* info) { return std::max(1, info->sm_count / 2); }
+
 size_t partial_bytes(int n, int splits) {
-  return static_cast<size_t>(splits) * tiles_for(n) * kBM * kBNMax * sizeof(float);
+  return static_cast<size_t>(splits) * tiles_for(n) * kTile * kTile * sizeof(float);
 }
 
 size_t diag_bytes(int n, int64_t n_tok) {
@@ -377,7 +372,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 size_t hessian_workspace_size(int n, int64_t n_tok) {
   const DeviceInfo* info = device_info();
   if (info == nullptr || n <= 0 || n_tok <= 0) return 0;
-  const int splits = choose_splits(n, n_tok, info->sm_count);
+  const int splits = choose_splits(n, n_tok, pairs_for(info));
   return align256(partial_bytes(n, splits)) + align256(diag_bytes(n, n_tok));
 }
 
@@ -386,7 +381,7 @@ gptq_status hessian_accum(float* H, double* hdiag, const void* X, int64_t n_tok,
   const DeviceInfo* info = device_info();
   if (info == nullptr) return GPTQ_ERR_CUDA;
   if (n_tok == 0) return GPTQ_OK;
-  const int splits = choose_splits(n, n_tok, info->sm_count);
+  const int splits = choose_splits(n, n_tok, pairs_for(info));
   const size_t pbytes = align256(partial_bytes(n, splits));
   if (ws_bytes < pbytes + align256(diag_bytes(n, n_tok))) return GPTQ_ERR_INVALID_ARG;
   float* partial = static_cast<float*>(ws);
@@ -415,10 +410,22 @@ gptq_status hessian_accum(float* H, double* hdiag, const void* X, int64_t n_tok,
   p.status = info->status;
   p.wait_ns = wait_limit_ns();
   const int units = p.splits * p.tiles;
-  const int grid = std::min(info->sm_count, units);
-  launch(syrk_tc_kernel, grid, kThreads, kSmemBytes, stream, xmap, p);
-  if (launch_status() != GPTQ_OK) return GPTQ_ERR_CUDA;
-  launch(syrk_finalize_kernel, dim3(p.tiles, kBNMax / 32, kBM / 32), dim3(32, 8), 0, stream, partial, H, n, p.tiles,
+  const int pairs = std::min(pairs_for(info), units);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, syrk_tc_kernel, xmap, p) != cudaSuccess) return GPTQ_ERR_CUDA;
+  count_launch();
+  launch(syrk_finalize_kernel, dim3(p.tiles, kTile / 32, kTile / 32), dim3(32, 8), 0, stream, partial, H, n, p.tiles,
                                                                                         p.splits, alpha);
   if (launch_status() != GPTQ_OK) return GPTQ_ERR_CUDA;
 
