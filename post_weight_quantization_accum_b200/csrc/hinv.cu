@@ -122,6 +122,7 @@ __global__ void gather_reversed_kernel(const float* __restrict__ H, const int32_
 
 constexpr int kPad = 68;           // shared-memory row stride (16-byte aligned rows)
 constexpr int kCholThreads = 256;
+constexpr int kMaxCholCtas = 4096;  // bound on the cooperative grid (SM ids recorded per CTA)
 constexpr size_t kCholSmem = 3 * kT * kPad * sizeof(float);
 
 struct CholArgs {
@@ -134,6 +135,7 @@ struct CholArgs {
   int* abort;        // set when a barrier wait runs out (zeroed on entry)
   uint64_t wait_ns;
   int vec;           // n % 4 == 0: rows of four along a tile row are 16-byte aligned
+  unsigned* smids;   // [gridDim.x] SM of each CTA
 };
 
 typedef float Tile[kPad];
@@ -500,18 +502,41 @@ __device__ void run_phase(const CholArgs& p, int k, int t0, int step, int total,
   }
 }
 
+__device__ __forceinline__ unsigned sm_id() {
+  unsigned r;
+  asm volatile("mov.u32 %0, %%smid;" : "=r"(r));
+  return r;
+}
+
 __global__ void __launch_bounds__(kCholThreads, 2) chol_inv_kernel(CholArgs p) {
   extern __shared__ __align__(16) float chol_smem[];
+  __shared__ int sib_s;
   Tile* s0 = reinterpret_cast<Tile*>(chol_smem);
   Tile* s1 = s0 + kT;
   Tile* s2 = s1 + kT;
   const int nb = p.nblk;
   const int G = static_cast<int>(gridDim.x), b = static_cast<int>(blockIdx.x);
+  // Every CTA records its SM; the CTA that shares CTA 0's SM (if any) takes no
+  // tile operations, so the diagonal factorizations (the kernel's critical
+  // path, run by CTA 0) have their SM to themselves.
+  if (threadIdx.x == 0) p.smids[b] = sm_id();
+  if (threadIdx.x == 0) sib_s = -1;
   if (b == 0) factor_diag(p, 0, s0, s1, s2);
   if (!grid_sync(p)) return;
+  {
+    const unsigned sm0 = __ldcg(p.smids);
+    for (int c = 1 + threadIdx.x; c < G; c += blockDim.x)
+      if (__ldcg(p.smids + c) == sm0) atomicMax(&sib_s, c);
+    __syncthreads();
+  }
+  const int sib = sib_s;
+  const bool idle = (b == sib);
+  const int pidx = b - ((sib >= 0 && b > sib) ? 1 : 0);  // index among the CTAs that work
+  const int PT = G - (sib >= 0 ? 1 : 0);
+  const int W = PT - 1;                                    // workers besides CTA 0
   for (int k = 0; k < nb; ++k) {
     // phase T(k): trsm of panel k and row k of the inverse
-    run_phase<false>(p, k, b, G, nb - 1, s0, s1, s2);
+    if (!idle) run_phase<false>(p, k, pidx, PT, nb - 1, s0, s1, s2);
     if (!grid_sync(p)) return;
     // phase U(k): CTA 0 updates tile (k+1, k+1) and then factors it; the
     // other CTAs share the remaining updates, so the factorization is the only
@@ -519,12 +544,13 @@ __global__ void __launch_bounds__(kCholThreads, 2) chol_inv_kernel(CholArgs p) {
     // pipelined loop, where no prefetched operands are live.
     const int m = nb - k - 1;
     const int total = m * (m + 1) / 2 + m * (k + 1);
-    if (G == 1)
-      run_phase<true>(p, k, 0, 1, total, s0, s1, s2);
-    else if (b == 0)
+    if (W == 0) {
+      if (b == 0) run_phase<true>(p, k, 0, 1, total, s0, s1, s2);
+    } else if (b == 0) {
       run_phase<true>(p, k, 0, total, total, s0, s1, s2);
-    else
-      run_phase<true>(p, k, b, G - 1, total, s0, s1, s2);
+    } else if (!idle) {
+      run_phase<true>(p, k, pidx, W, total, s0, s1, s2);
+    }
     if (b == 0 && m > 0) factor_diag(p, k + 1, s0, s1, s2);
     if (!grid_sync(p)) return;
   }
@@ -548,8 +574,8 @@ PrepLayout prep_layout(int n) {
   off += align256(static_cast<size_t>(n));
   l.lambda = off;
   off += 256;
-  l.bar = off;  // barrier words and the abort flag
-  off += 256;
+  l.bar = off;  // barrier words and the abort flag, then one SM id per CTA
+  off += 256 + align256(kMaxCholCtas * sizeof(unsigned));
   l.perm = off;
   off += align256(static_cast<size_t>(n) * sizeof(int32_t));
   l.total = off;
@@ -565,7 +591,7 @@ int chol_grid(const DeviceInfo* info) {
       return 0;
     blocks_per_sm[info->device] = std::min(b, 2);
   }
-  return blocks_per_sm[info->device] * info->sm_count;
+  return std::min(kMaxCholCtas, blocks_per_sm[info->device] * info->sm_count);
 }
 
 }  // namespace
@@ -619,6 +645,7 @@ gptq_status prepare_hinv(const float* H, const double* hdiag, int n, float damp,
   ca.fstatus = fstatus;
   ca.bar = bar;
   ca.abort = reinterpret_cast<int*>(bar + 2);
+  ca.smids = bar + 64;
   ca.wait_ns = wait_limit_ns();
   ca.vec = (n % 4 == 0) ? 1 : 0;
   void* args[] = {&ca};

@@ -185,6 +185,28 @@ def test_prepare_matches_oracle(n, act_order):
         assert np.linalg.norm(r) / np.linalg.norm(v) <= 1e-3
 
 
+def test_factorization_wait_timeout_is_reported_and_recoverable():
+    """A made-to-run-out wait: with the in-kernel wait bound at 0 ns the first
+    CTA that has to wait at a grid barrier of the factorization gives up, sets
+    the abort flag and every CTA returns; the call reports GPTQ_ERR_TIMEOUT and
+    the next call on the same context succeeds.  (The factorization kernel has
+    no asynchronous copies or tensor memory, so nothing is left in flight.)"""
+    n = 512
+    X, Hx = _spd_from_x(n, 4 * n, seed=77)
+    H32 = torch.tensor(Hx.astype(np.float32), device="cuda")
+    try:
+        gq.gptq_set_wait_limit_ns(0)
+        with pytest.raises(gq.GptqError) as ei:
+            gq.gptq_prepare_hinv(H32.clone(), 0.01, False)
+        assert ei.value.status == "GPTQ_ERR_TIMEOUT"
+    finally:
+        gq.gptq_set_wait_limit_ns(2 ** 64 - 1)
+    U, perm, dead = gq.gptq_prepare_hinv(H32.clone(), 0.01, False)
+    torch.cuda.synchronize()
+    prep = go.prepare(Hx.astype(np.float32).astype(np.float64), np.zeros((1, n)), 0.01, False)
+    assert rel_fro(np64(U), go.inverse_factor(prep["H"])) <= 1e-4
+
+
 def test_prepare_not_positive_definite():
     n = 96
     g = torch.Generator(device="cuda").manual_seed(1)
