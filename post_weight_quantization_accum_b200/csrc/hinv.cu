@@ -143,9 +143,6 @@ typedef float Tile[kPad];
 __device__ __forceinline__ float ld_a(const CholArgs& p, int r, int c) {
   return (r < p.n && c < p.n) ? __ldcg(p.A + static_cast<size_t>(r) * p.n + c) : 0.0f;
 }
-__device__ __forceinline__ float ld_x(const CholArgs& p, int r, int c) {
-  return (r < p.n && c < p.n) ? __ldcg(p.U + static_cast<size_t>(p.n - 1 - r) * p.n + (p.n - 1 - c)) : 0.0f;
-}
 __device__ __forceinline__ float* at_a(const CholArgs& p, int r, int c) { return p.A + static_cast<size_t>(r) * p.n + c; }
 __device__ __forceinline__ float* at_x(const CholArgs& p, int r, int c) {
   return p.U + static_cast<size_t>(p.n - 1 - r) * p.n + (p.n - 1 - c);
@@ -367,6 +364,38 @@ __device__ __forceinline__ void st4(const CholArgs& p, bool to_x, int r, int c, 
   }
 }
 
+// Adds v to four consecutive entries (r, c .. c + 3) of A or X in memory (a
+// reduction performed in L2: no read into the SM, nothing to wait for).
+// Each entry receives one such addition per phase, so the result is that of
+// a load, an fp32 addition and a store.
+__device__ __forceinline__ void red4(const CholArgs& p, bool to_x, int r, int c, float4 v) {
+  if (r >= p.n || c >= p.n) return;
+  if (!to_x) {
+    float* dst = p.A + static_cast<size_t>(r) * p.n + c;
+    if (p.vec) {
+      asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+                   : "memory");
+    } else {
+      atomicAdd(dst, v.x);
+      if (c + 1 < p.n) atomicAdd(dst + 1, v.y);
+      if (c + 2 < p.n) atomicAdd(dst + 2, v.z);
+      if (c + 3 < p.n) atomicAdd(dst + 3, v.w);
+    }
+  } else {
+    float* row = p.U + static_cast<size_t>(p.n - 1 - r) * p.n + (p.n - 1);
+    if (p.vec) {
+      asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(row - c - 3), "f"(v.w), "f"(v.z), "f"(v.y),
+                   "f"(v.x)
+                   : "memory");
+    } else {
+      atomicAdd(row - c, v.x);
+      if (c + 1 < p.n) atomicAdd(row - c - 1, v.y);
+      if (c + 2 < p.n) atomicAdd(row - c - 2, v.z);
+      if (c + 3 < p.n) atomicAdd(row - c - 3, v.w);
+    }
+  }
+}
+
 // Which four entries (row a, columns 4 b4 .. 4 b4 + 3) of a 64 x 64 operand
 // thread t stages in its slot g.  An operand that shared memory keeps
 // transposed uses mapping T: two lanes per row (one 32-byte sector per row and
@@ -384,16 +413,15 @@ __device__ __forceinline__ void slot_n(int g, int& a, int& b4) {
   b4 = idx & 15;
 }
 
-// Registers holding one tile operation's operands (and, for the subtracting
-// operations, the old output values) between its loads and its use.
+// Registers holding one tile operation's operands between their loads and
+// their use.
 struct Staged {
-  float4 p[4], q[4], o[4];
+  float4 p[4], q[4];
 };
 
 __device__ __forceinline__ bool q_natural(const TileOp& op) { return op.kind == kOpFinalize || op.kind == kOpInverse; }
 
 __device__ __forceinline__ void fetch_op(const CholArgs& p, const TileOp& op, int k0, Staged& st) {
-  const int tr = (threadIdx.x / 16) * 4, tc = (threadIdx.x % 16) * 4;
 #pragma unroll
   for (int g = 0; g < 4; ++g) {
     int a, b4, an, bn4;
@@ -418,12 +446,6 @@ __device__ __forceinline__ void fetch_op(const CholArgs& p, const TileOp& op, in
         st.q[g] = ld4_x(p, k0 + an, op.j0 + 4 * bn4);
         break;
     }
-  }
-  if (op.kind == kOpUpdate || op.kind == kOpInverse) {
-    const bool to_x = op.kind == kOpInverse;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      st.o[i] = to_x ? ld4_x(p, op.i0 + tr + i, op.j0 + tc) : ld4_a(p, op.i0 + tr + i, op.j0 + tc);
   }
 }
 
@@ -453,8 +475,9 @@ __device__ __forceinline__ void commit_op(const TileOp& op, const Staged& st, Ti
   }
 }
 
-__device__ __forceinline__ void finish_op(const CholArgs& p, const TileOp& op, int k0, const float (&acc)[4][4],
-                                          const float4* old) {
+// Writes the product (trsm, finalize) or subtracts it in place (update,
+// inverse: an L2 reduction, so the old values never travel to the SM).
+__device__ __forceinline__ void finish_op(const CholArgs& p, const TileOp& op, int k0, const float (&acc)[4][4]) {
   const int tr = (threadIdx.x / 16) * 4, tc = (threadIdx.x % 16) * 4;
   const bool to_x = op.kind == kOpFinalize || op.kind == kOpInverse;
   const bool subtract = op.kind == kOpUpdate || op.kind == kOpInverse;
@@ -462,12 +485,10 @@ __device__ __forceinline__ void finish_op(const CholArgs& p, const TileOp& op, i
   const int c0 = op.kind == kOpTrsm ? k0 : op.j0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    float4 v = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
-    if (subtract) {
-      const float4 o = old[i * kCholThreads];
-      v = make_float4(o.x - v.x, o.y - v.y, o.z - v.z, o.w - v.w);
-    }
-    st4(p, to_x, r0 + tr + i, c0 + tc, v);
+    if (subtract)
+      red4(p, to_x, r0 + tr + i, c0 + tc, make_float4(-acc[i][0], -acc[i][1], -acc[i][2], -acc[i][3]));
+    else
+      st4(p, to_x, r0 + tr + i, c0 + tc, make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]));
   }
 }
 
@@ -475,7 +496,7 @@ __device__ __forceinline__ void finish_op(const CholArgs& p, const TileOp& op, i
 // the next operation are loaded into registers while the current one is
 // multiplied, so L2 latency overlaps the FMAs.
 template <bool kPhaseU>
-__device__ void run_phase(const CholArgs& p, int k, int t0, int step, int total, Tile* s0, Tile* s1, Tile* s2) {
+__device__ void run_phase(const CholArgs& p, int k, int t0, int step, int total, Tile* s0, Tile* s1) {
   if (t0 >= total) return;
   const int nb = p.nblk, k0 = k * kT;
   Staged st;
@@ -483,10 +504,6 @@ __device__ void run_phase(const CholArgs& p, int k, int t0, int step, int total,
   fetch_op(p, cur, k0, st);
   for (int t = t0; t < total; t += step) {
     commit_op(cur, st, s0, s1);
-    // the old output values wait in s2 (float4 slot [i][thread], conflict-free)
-    float4* old = reinterpret_cast<float4*>(&s2[0][0]) + threadIdx.x;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) old[i * kCholThreads] = st.o[i];
     __syncthreads();
     const int tn = t + step;
     TileOp nxt = cur;
@@ -496,10 +513,12 @@ __device__ void run_phase(const CholArgs& p, int k, int t0, int step, int total,
     }
     float acc[4][4];
     tile_product(s0, s1, acc);
-    finish_op(p, cur, k0, acc, old);
+    finish_op(p, cur, k0, acc);
     __syncthreads();
     cur = nxt;
   }
+  __threadfence();  // this CTA's reductions are performed before its later reads
+  __syncthreads();
 }
 
 __device__ __forceinline__ unsigned sm_id() {
@@ -536,7 +555,7 @@ __global__ void __launch_bounds__(kCholThreads, 2) chol_inv_kernel(CholArgs p) {
   const int W = PT - 1;                                    // workers besides CTA 0
   for (int k = 0; k < nb; ++k) {
     // phase T(k): trsm of panel k and row k of the inverse
-    if (!idle) run_phase<false>(p, k, pidx, PT, nb - 1, s0, s1, s2);
+    if (!idle) run_phase<false>(p, k, pidx, PT, nb - 1, s0, s1);
     if (!grid_sync(p)) return;
     // phase U(k): CTA 0 updates tile (k+1, k+1) and then factors it; the
     // other CTAs share the remaining updates, so the factorization is the only
@@ -545,11 +564,11 @@ __global__ void __launch_bounds__(kCholThreads, 2) chol_inv_kernel(CholArgs p) {
     const int m = nb - k - 1;
     const int total = m * (m + 1) / 2 + m * (k + 1);
     if (W == 0) {
-      if (b == 0) run_phase<true>(p, k, 0, 1, total, s0, s1, s2);
+      if (b == 0) run_phase<true>(p, k, 0, 1, total, s0, s1);
     } else if (b == 0) {
-      run_phase<true>(p, k, 0, total, total, s0, s1, s2);
+      run_phase<true>(p, k, 0, total, total, s0, s1);
     } else if (!idle) {
-      run_phase<true>(p, k, pidx, W, total, s0, s1, s2);
+      run_phase<true>(p, k, pidx, W, total, s0, s1);
     }
     if (b == 0 && m > 0) factor_diag(p, k + 1, s0, s1, s2);
     if (!grid_sync(p)) return;
