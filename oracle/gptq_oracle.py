@@ -81,6 +81,7 @@ __all__ = [
     "pack_codes",
     "unpack_codes",
     "packed_words_per_row",
+    "dequant_matvec",
 ]
 
 
@@ -477,3 +478,26 @@ def unpack_codes(packed, n, bits):
     stream = (packed[:, :, None] >> np.arange(32)) & 1               # [rows, words, 32]
     stream = stream.reshape(rows, words * 32)[:, : n * bits].reshape(rows, n, bits)
     return np.sum(stream << np.arange(bits), axis=2).astype(np.int64)
+
+
+# ---------------------------------------------------------------------------
+# Inference with the packed weights (GPTQ abstract on the "Daily Papers" page:
+# the packed 3/4-bit weights run generative inference faster than FP16; GPTQ
+# knowledge note, "Tradeoffs": deployment reads packed weights)
+# ---------------------------------------------------------------------------
+
+def dequant_matvec(packed, scales, zeros, n, bits, group, x, g_idx=None):
+    """y[b, r] = sum_c Q[r, c] * x[b, c] for the dequantized weights
+    Q[r, c] = scales[r, g(c)] * (code[r, c] - zeros[r, g(c)]), where the codes
+    are read back from the packed rows (original column order) and g(c) is
+    g_idx[c] when given (act-order) else c // group (group 0: one group per
+    row).  x is [batch, n]; fp64 throughout."""
+    codes = unpack_codes(packed, n, bits).astype(np.float64)
+    rows = codes.shape[0]
+    G = group if group > 0 else max(n, 1)
+    g = np.asarray(g_idx, dtype=np.int64) if g_idx is not None else np.arange(n) // G
+    s = np.asarray(scales, dtype=np.float64)[:, g]
+    z = np.asarray(zeros, dtype=np.float64)[:, g]
+    Q = s * (codes - z)
+    x = np.atleast_2d(np.asarray(x, dtype=np.float64))
+    return x @ Q.T

@@ -31,6 +31,9 @@ MUTATIONS = {
     "damping from max": ("lam = float(damp) * float(np.mean(np.diag(H)))", "lam = float(damp) * float(np.max(np.diag(H)))"),
     "lower factor instead of upper": ("return _cholesky(Hinv).T", "return _cholesky(Hinv)"),
     "reversed factor not reversed back": ("return _lower_inverse(Lr)[::-1, ::-1].copy()", "return _lower_inverse(Lr).T.copy()"),
+    "matvec groups interleaved": ("else np.arange(n) // G", "else np.arange(n) % max(n // G, 1)"),
+    "matvec zero point added": ("Q = s * (codes - z)", "Q = s * (codes + z)"),
+    "matvec transposed product": ("return x @ Q.T", "return (Q @ x.T).T[:, ::-1]"),
 }
 
 
@@ -137,7 +140,16 @@ def _pin_diag_rtn(go):
     assert np.array_equal(out["codes"], ref["codes"])
 
 
-PINS = [_pin_worked_examples, _pin_grid, _pin_block_invariance, _pin_identities, _pin_babai, _pin_diag_rtn]
+def _pin_matvec(go):
+    for case in _golden("matvec_examples.json")["cases"]:
+        packed = np.array([[int(w, 16) for w in row] for row in case["packed"]], dtype=np.uint32)
+        y = go.dequant_matvec(packed, np.array(case["scales"]), np.array(case["zeros"]), case["n"], case["bits"],
+                              case["group"], np.array(case["x"]), case.get("g_idx"))
+        assert np.array_equal(y, np.array(case["y"]))
+
+
+PINS = [_pin_worked_examples, _pin_grid, _pin_block_invariance, _pin_identities, _pin_babai, _pin_diag_rtn,
+        _pin_matvec]
 
 
 def test_pins_pass_on_the_oracle():

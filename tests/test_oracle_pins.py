@@ -124,6 +124,32 @@ def test_pack_roundtrip(bits, n):
     assert go.packed_words_per_row(32 * 7, bits) * 32 == 32 * 7 * bits
 
 
+def test_dequant_matvec_examples(golden_dir):
+    """Hand-derived packed matvec cases, natural groups and an act-order g_idx."""
+    for case in _cases(golden_dir, "matvec_examples.json")["cases"]:
+        packed = np.array([[int(w, 16) for w in row] for row in case["packed"]], dtype=np.uint32)
+        y = go.dequant_matvec(packed, np.array(case["scales"]), np.array(case["zeros"]), case["n"], case["bits"],
+                              case["group"], np.array(case["x"]), case.get("g_idx"))
+        assert np.array_equal(y, np.array(case["y"]))
+
+
+@pytest.mark.parametrize("act_order", [False, True])
+@pytest.mark.parametrize("bits,group", [(4, 32), (3, 0), (2, 16)])
+def test_dequant_matvec_matches_layer_dequantized_weights(act_order, bits, group):
+    """Reading the codes back from the packed stream and applying the grid per
+    g_idx reproduces the column loop's own dequantized weights (computed along
+    a different path, inside the loop), so the matvec equals deq @ x."""
+    rng = np.random.default_rng(3 + bits)
+    rows, n = 5, 64
+    X = rng.standard_normal((200, n)) * np.exp(rng.standard_normal(n))
+    W = rng.standard_normal((rows, n)) * 0.02
+    ref = go.gptq_layer(W, X=X, bits=bits, group=group, block=32, act_order=act_order)
+    x = rng.standard_normal((3, n))
+    y = go.dequant_matvec(go.pack_codes(ref["codes"], bits), ref["scales"], ref["zeros"], n, bits, group, x,
+                          ref["g_idx"] if act_order else None)
+    np.testing.assert_allclose(y, x @ ref["deq"].T, rtol=1e-12, atol=1e-14)
+
+
 # ---------------------------------------------------------------------------
 # Hessian
 # ---------------------------------------------------------------------------
