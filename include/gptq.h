@@ -268,6 +268,43 @@ int32_t gptq_packed_words_per_row(int32_t n, int32_t bits);
 gptq_status gptq_pack(const uint8_t* codes, int64_t rows, int32_t n, int32_t bits,
                       uint32_t* packed, void* stream);
 
+/* ------------------------------------------------------------------------ */
+/* 5. Inference with the packed weights                                      */
+/* ------------------------------------------------------------------------ */
+
+/* Bytes of workspace gptq_dequant_matvec needs: 0 in this version (x is read
+ * in place in either dtype); kept so that callers size it the usual way. */
+size_t gptq_matvec_workspace_size(int32_t n, int32_t batch, gptq_dtype xdt);
+
+/* y[b, r] = sum_c Q[r, c] * x[b, c] for b < batch, r < rows, where
+ * Q[r, c] = scales[r, g(c)] * (code[r, c] - zeros[r, g(c)]) is read straight
+ * from the packed rows; g(c) = g_idx[c] when g_idx is given (act-order), else
+ * c / group (group 0: one group per row).
+ *
+ * Source: the GPTQ abstract on the "Daily Papers" page (the packed 3/4-bit
+ * weights run generative inference faster than FP16) and the GPTQ knowledge
+ * note, "Tradeoffs" (deployment reads packed weights).  The arithmetic is the
+ * grid's dequantization (scale * (code - zero)) applied to the packed format
+ * of gptq_pack.
+ *
+ *   packed   uint32 [rows, gptq_packed_words_per_row(n, bits)], codes in
+ *            ORIGINAL column order (as gptq_quantize_layer returns them, then
+ *            gptq_pack), 4-byte aligned
+ *   scales   fp32 [rows, n_groups]; zeros uint8 [rows, n_groups]
+ *   g_idx    int32 [n] group of each original column, or NULL
+ *   x        [batch, n] (xdt = GPTQ_F32 or GPTQ_BF16), 1 <= batch <= 8
+ *   y        fp32 [batch, rows], written
+ *   ws       gptq_matvec_workspace_size(n, batch, xdt) bytes (256-byte aligned;
+ *            may be NULL when that is 0, as it is in this version)
+ * Accumulates in fp32.  Asynchronous on `stream`.
+ * Errors: GPTQ_ERR_INVALID_ARG (sizes, bits not in {2,3,4,8}, group > n,
+ * batch outside 1..8, NULL or misaligned pointers, small workspace), before any
+ * launch; GPTQ_ERR_CUDA. */
+gptq_status gptq_dequant_matvec(const uint32_t* packed, const float* scales, const uint8_t* zeros,
+                                const int32_t* g_idx, int64_t rows, int32_t n, int32_t bits, int32_t group,
+                                const void* x, gptq_dtype xdt, int32_t batch, float* y, void* ws,
+                                size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -18,6 +18,7 @@ __all__ = [
     "gptq_quantize_layer",
     "gptq_quantize_rtn",
     "gptq_pack",
+    "gptq_dequant_matvec",
     "gptq_get_device_status",
     "gptq_set_wait_limit_ns",
     "gptq_kernel_launches",
@@ -143,6 +144,27 @@ def gptq_pack(codes, bits, packed=None, stream=None):
         packed = torch.empty((rows, words), dtype=torch.int32, device=codes.device)
     check("gptq_pack", LIB.gptq_pack(_ptr(codes), rows, n, bits, _ptr(packed), _stream(stream)))
     return packed
+
+
+def gptq_dequant_matvec(packed, scales, zeros, n, bits, group, x, g_idx=None, y=None, ws=None, stream=None):
+    """y[b, r] = sum_c Q[r, c] x[b, c] with Q read from the packed rows; x is
+    [batch, n] (or [n]) fp32 or bf16 on the device; returns fp32 [batch, rows]."""
+    rows = packed.shape[0]
+    squeeze = x.dim() == 1
+    x2 = x.reshape(1, -1) if squeeze else x
+    batch = x2.shape[0]
+    xdt = _dtype_code(x2)
+    if y is None:
+        y = torch.empty((batch, rows), dtype=torch.float32, device=packed.device)
+    need = LIB.gptq_matvec_workspace_size(n, batch, xdt)
+    wp, wb = ctypes.c_void_p(0), 0
+    if need > 0:
+        wp, wb = _ws_ptr(ws if ws is not None else workspace(need, packed.device))
+    x2 = x2.contiguous()
+    check("gptq_dequant_matvec", LIB.gptq_dequant_matvec(_ptr(packed), _ptr(scales), _ptr(zeros), _ptr(g_idx), rows,
+                                                         n, bits, group, _ptr(x2), xdt, batch, _ptr(y), wp, wb,
+                                                         _stream(stream)))
+    return y[0] if squeeze else y
 
 
 def quantize_layer(W, X, bits=4, group=128, damp=0.01, block=128, act_order=False, want_deq=False,

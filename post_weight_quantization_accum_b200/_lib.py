@@ -46,6 +46,10 @@ _SIGS = {
                                          ctypes.c_int32, _P, _P, _P, _P]),
     "gptq_packed_words_per_row": (ctypes.c_int32, [ctypes.c_int32, ctypes.c_int32]),
     "gptq_pack": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, _P, _P]),
+    "gptq_matvec_workspace_size": (ctypes.c_size_t, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int]),
+    "gptq_dequant_matvec": (ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                                           ctypes.c_int32, _P, ctypes.c_int, ctypes.c_int32, _P, _P,
+                                           ctypes.c_size_t, _P]),
 }
 
 

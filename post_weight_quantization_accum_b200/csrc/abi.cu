@@ -1,5 +1,5 @@
 // C ABI of the library: argument validation, per-device state and dispatch to
-// the kernels in hessian.cu, hinv.cu, quantize.cu and pack.cu.  Nothing here
+// the kernels in hessian.cu, hinv.cu, quantize.cu, pack.cu and matvec.cu.  Nothing here
 // allocates device memory; every scratch byte comes from the caller.
 #include <atomic>
 #include <cmath>
@@ -24,6 +24,10 @@ gptq_status quantize_layer(const void* W, gptq_dtype wdt, int64_t rows, int n, c
 gptq_status quantize_rtn(const void* W, gptq_dtype wdt, int64_t rows, int n, int bits, int group, uint8_t* codes,
                          float* scales, uint8_t* zeros, cudaStream_t st);
 gptq_status pack_codes(const uint8_t* codes, int64_t rows, int n, int bits, uint32_t* packed, cudaStream_t st);
+size_t matvec_workspace_size(int n, int batch, int xdt_bf16);
+gptq_status dequant_matvec(const uint32_t* packed, const float* scales, const uint8_t* zeros, const int32_t* g_idx,
+                           int64_t rows, int n, int bits, int group, const void* x, int xdt_bf16, int batch, float* y,
+                           void* ws, cudaStream_t st);
 
 // Status words of each device: [0] failures of asynchronous kernels (bounded
 // waits), [1] the factorization status of gptq_prepare_hinv.
@@ -216,6 +220,29 @@ gptq_status gptq_pack(const uint8_t* codes, int64_t rows, int32_t n, int32_t bit
   if (rows == 0) return GPTQ_OK;
   if (codes == nullptr || packed == nullptr || !aligned(packed, 4)) return GPTQ_ERR_INVALID_ARG;
   return pack_codes(codes, rows, n, bits, packed, as_stream(stream));
+}
+
+size_t gptq_matvec_workspace_size(int32_t n, int32_t batch, gptq_dtype xdt) {
+  if (n < 1 || batch < 1) return 0;
+  return matvec_workspace_size(n, batch, xdt == GPTQ_BF16 ? 1 : 0);
+}
+
+gptq_status gptq_dequant_matvec(const uint32_t* packed, const float* scales, const uint8_t* zeros,
+                                const int32_t* g_idx, int64_t rows, int32_t n, int32_t bits, int32_t group,
+                                const void* x, gptq_dtype xdt, int32_t batch, float* y, void* ws, size_t ws_bytes,
+                                void* stream) {
+  if (rows < 0 || n < 1 || n > kMaxN || !valid_bits(bits) || group < 0 || group > n || batch < 1 || batch > 8 ||
+      (xdt != GPTQ_F32 && xdt != GPTQ_BF16))
+    return GPTQ_ERR_INVALID_ARG;
+  if (rows == 0) return GPTQ_OK;
+  if (packed == nullptr || scales == nullptr || zeros == nullptr || x == nullptr || y == nullptr ||
+      !aligned(packed, 4) || !aligned(scales, 4) || !aligned(y, 4) || !aligned(x, xdt == GPTQ_BF16 ? 2 : 4) ||
+      (g_idx != nullptr && !aligned(g_idx, 4)))
+    return GPTQ_ERR_INVALID_ARG;
+  const size_t need = matvec_workspace_size(n, batch, xdt == GPTQ_BF16 ? 1 : 0);
+  if (need > 0 && (ws == nullptr || !aligned(ws, 256) || ws_bytes < need)) return GPTQ_ERR_INVALID_ARG;
+  return dequant_matvec(packed, scales, zeros, g_idx, rows, n, bits, group, x, xdt == GPTQ_BF16 ? 1 : 0, batch, y, ws,
+                        as_stream(stream));
 }
 
 }  // extern "C"
