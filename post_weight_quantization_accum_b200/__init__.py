@@ -167,25 +167,67 @@ def gptq_dequant_matvec(packed, scales, zeros, n, bits, group, x, g_idx=None, y=
     return y[0] if squeeze else y
 
 
+def _hessian_from_host(H, X, hdiag, stream, chunk_tokens):
+    """H += (2/N) X^T X for calibration inputs in host memory: token chunks are
+    copied into two device buffers on a copy stream while the library
+    accumulates the previous chunk, so the transfer and the SYRK overlap.
+    (Pinned host memory makes the copies asynchronous.)"""
+    n_tok, n = X.shape
+    dev = H.device
+    compute = stream if stream is not None else torch.cuda.current_stream(dev)
+    copy = torch.cuda.Stream(dev)
+    pitch = (n + 7) // 8 * 8
+    m = min(chunk_tokens, n_tok)
+    bufs = [torch.empty((m, pitch), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    ready = [torch.cuda.Event() for _ in range(2)]
+    free = [torch.cuda.Event() for _ in range(2)]
+    ws = workspace(LIB.gptq_hessian_workspace_size(n, m), dev)
+    ws.record_stream(compute)
+    alpha = 2.0 / n_tok
+    for i, t0 in enumerate(range(0, n_tok, m)):
+        k = i % 2
+        rows = min(m, n_tok - t0)
+        if i >= 2:
+            copy.wait_event(free[k])
+        with torch.cuda.stream(copy):
+            bufs[k][:rows, :n].copy_(X[t0:t0 + rows], non_blocking=True)
+            ready[k].record(copy)
+        compute.wait_event(ready[k])
+        gptq_hessian_accum(H, bufs[k][:rows, :n], alpha, hdiag=hdiag, ws=ws, stream=compute)
+        free[k].record(compute)
+        bufs[k].record_stream(compute)
+    return H
+
+
 def quantize_layer(W, X, bits=4, group=128, damp=0.01, block=128, act_order=False, want_deq=False,
-                   want_loss=False, stream=None):
+                   want_loss=False, stream=None, device=None, chunk_tokens=16384):
     """One linear layer end to end: H from X, U, the column loop, packing.
 
     W: [rows, n] fp32/bf16 weights; X: [n_tok, n] bf16 calibration inputs.
-    Returns a dict with H, U, perm, codes, scales, zeros, g_idx, packed,
-    packed_zeros (and deq / row_loss when asked for).
+    Either may live in host memory (ideally pinned): X is then streamed to the
+    GPU in chunks of `chunk_tokens` tokens, each chunk's SYRK overlapping the
+    copy of the next.  Everything is computed on `device` (default: W's device
+    if W is on a GPU, else the current one).  Returns a dict of device tensors
+    with H, U, perm, codes, scales, zeros, g_idx, packed, packed_zeros (and deq
+    / row_loss when asked for).
     """
     n = W.shape[1]
-    dev = W.device
-    if X.stride(1) != 1 or X.stride(0) % 8 != 0 or X.data_ptr() % 16 != 0:
-        # the library streams X with TMA, whose row pitch must be a multiple
-        # of 16 bytes: hand it a row-padded copy
-        Xp = torch.zeros((X.shape[0], (n + 7) // 8 * 8), dtype=torch.bfloat16, device=dev)
-        Xp[:, :n] = X
-        X = Xp[:, :n]
+    dev = torch.device(device) if device is not None else (W.device if W.is_cuda else
+                                                             torch.device("cuda", torch.cuda.current_device()))
+    if not W.is_cuda:
+        W = W.to(dev, non_blocking=True)
     H = torch.zeros((n, n), dtype=torch.float32, device=dev)
     hdiag = torch.zeros(n, dtype=torch.float64, device=dev) if act_order else None
-    gptq_hessian_accum(H, X, 2.0 / X.shape[0], hdiag=hdiag, stream=stream)
+    if not X.is_cuda:
+        _hessian_from_host(H, X, hdiag, stream, chunk_tokens)
+    else:
+        if X.stride(1) != 1 or X.stride(0) % 8 != 0 or X.data_ptr() % 16 != 0:
+            # the library streams X with TMA, whose row pitch must be a multiple
+            # of 16 bytes: hand it a row-padded copy
+            Xp = torch.zeros((X.shape[0], (n + 7) // 8 * 8), dtype=torch.bfloat16, device=dev)
+            Xp[:, :n] = X
+            X = Xp[:, :n]
+        gptq_hessian_accum(H, X, 2.0 / X.shape[0], hdiag=hdiag, stream=stream)
     U, perm, dead = gptq_prepare_hinv(H, damp, act_order, hdiag=hdiag, stream=stream)
     out = gptq_quantize_layer(W, U, bits, group, block, perm=perm if act_order else None, dead=dead,
                               want_deq=want_deq, want_loss=want_loss, stream=stream)

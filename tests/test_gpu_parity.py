@@ -311,6 +311,23 @@ def test_tiny_and_ragged_shapes():
         assert abs(err_gpu - err_ref) <= 1e-3 * max(err_ref, 1e-30) + 1e-12
 
 
+@pytest.mark.parametrize("n,act_order", [(256, False), (300, True)])
+def test_host_inputs_stream_in_chunks(n, act_order):
+    """quantize_layer with W and X in (pinned) host memory streams X in token
+    chunks; H equals the one-shot device H up to fp32 summation order, and the
+    codes agree with the device call."""
+    spec = si.scaled(si.SPECS["mlp_up" if act_order else "attn4096"], rows=48, n=n, n_tok=5000)
+    W, X = si.make_layer(spec, "cuda")
+    ref = gq.quantize_layer(W, X, bits=spec.bits, group=spec.group, act_order=act_order)
+    got = gq.quantize_layer(W.cpu().pin_memory(), X.cpu().pin_memory(), bits=spec.bits, group=spec.group,
+                            act_order=act_order, chunk_tokens=1024)
+    torch.cuda.synchronize()
+    assert rel_fro(np64(got["H"]), np64(ref["H"])) <= 1e-6
+    assert float((got["codes"] == ref["codes"]).float().mean()) >= 0.999
+    if act_order:
+        assert torch.equal(got["perm"], ref["perm"])
+
+
 def test_packed_outputs_roundtrip():
     spec = si.scaled(si.SPECS["attn4096"], rows=16, n=256, n_tok=1024, bits=3)
     W, X = si.make_layer(spec, "cuda")
