@@ -6,8 +6,23 @@
 // inverse of H):
 //
 //   A = J P^T (H + lambda I) P J          (J = order reversal, P = act-order)
-//   A = L L^T,  X = L^-1                  one persistent cooperative kernel
-//   U = J X J                             (X is stored rotated as it is made)
+//   A = L L^T,  X = L^-1                  blocked, see below
+//   U = J X J                             (a reversal of X's storage)
+//
+// Below n = 8192 one persistent cooperative kernel factors A and builds X in
+// 64-wide panels on the CUDA cores.  From there on the same kernel handles
+// each 1024 x 1024 diagonal block, and everything between blocks is a
+// tensor-core GEMM with the fp32-accurate 3-term tf32 split (trailing.cu):
+// for block K (rows and columns [k0, k1)), R the rows of X still being
+// formed,
+//   X_K,<K  = X_KK R_K,<K                 finalize block row K of X
+//   L_>K,K  = A_>K,K X_KK^T               panel (trsm as a product)
+//   A_>K,>K -= L_>K,K L_>K,K^T            trailing update (full square, which
+//                                         also keeps the diagonal tiles' upper
+//                                         halves the factorization reads)
+//   R_>K,<=K -= L_>K,K X_K,<=K            inverse update
+// so the O(n^3) work runs at tensor-core rate and only the 1024-wide diagonal
+// blocks go through the latency-bound panel sweep.
 //
 // With H' = P^T (H + lambda I) P, J H' J = L L^T gives H' = (J L J)(J L J)^T
 // with J L J upper triangular, so U = (J L J)^-1 = J L^-1 J is upper with
@@ -100,6 +115,18 @@ __global__ void gather_reversed_kernel(const float* __restrict__ H, const int32_
   A[static_cast<size_t>(a) * n + b] = v;
 }
 
+// U = J X J for X stored row-major in U's own memory: U[a][b] = X[n-1-a][n-1-b]
+// is the reversal of the flat array (element e <-> n*n - 1 - e).
+__global__ void reverse_kernel(float* __restrict__ U, int64_t count) {
+  const int64_t half = count / 2;
+  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < half;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float a = U[e], b = U[count - 1 - e];
+    U[e] = b;
+    U[count - 1 - e] = a;
+  }
+}
+
 // --------------------------------------------------------------------------
 // Cholesky and inverse in one persistent cooperative kernel
 // --------------------------------------------------------------------------
@@ -116,9 +143,9 @@ __global__ void gather_reversed_kernel(const float* __restrict__ H, const int32_
 //
 // Every step is a 64 x 64 x 64 tile product, and the Cholesky half of a phase
 // shrinks as the inverse half grows, so each phase has about the same number
-// of tiles.  Two grid barriers per panel (time-bounded).  X is written straight
-// into U's rotated position (U = J X J), so no rotation pass is needed;
-// R's tiles live in the same places before they are finalized.
+// of tiles.  Two grid barriers per panel (time-bounded).  The kernel works on
+// one diagonal block of order <= 1024 at any row pitch; R's tiles live in X's
+// places before they are finalized.
 
 constexpr int kPad = 68;           // shared-memory row stride (16-byte aligned rows)
 constexpr int kCholThreads = 256;
@@ -126,27 +153,26 @@ constexpr int kMaxCholCtas = 4096;  // bound on the cooperative grid (SM ids rec
 constexpr size_t kCholSmem = 3 * kT * kPad * sizeof(float);
 
 struct CholArgs {
-  float* A;          // [n, n] lower: the damped reversed matrix, becomes L
-  float* U;          // [n, n] zeroed on entry; X = L^-1 is written rotated
-  int n;
+  float* A;          // block [n, n] at row pitch lda, lower: the damped reversed matrix, becomes L
+  float* X;          // block [n, n] at row pitch ldx, zero on entry: X = L^-1 is written here
+  int64_t lda, ldx;
+  int n;             // order of the block
   int nblk;
   int* fstatus;      // factorization status word
   unsigned* bar;     // grid barrier: [0] arrivals, [1] generation (zeroed on entry)
   int* abort;        // set when a barrier wait runs out (zeroed on entry)
   uint64_t wait_ns;
-  int vec;           // n % 4 == 0: rows of four along a tile row are 16-byte aligned
+  int vec;           // rows of four along a tile row are 16-byte aligned (lda, ldx, bases)
   unsigned* smids;   // [gridDim.x] SM of each CTA
 };
 
 typedef float Tile[kPad];
 
 __device__ __forceinline__ float ld_a(const CholArgs& p, int r, int c) {
-  return (r < p.n && c < p.n) ? __ldcg(p.A + static_cast<size_t>(r) * p.n + c) : 0.0f;
+  return (r < p.n && c < p.n) ? __ldcg(p.A + r * p.lda + c) : 0.0f;
 }
-__device__ __forceinline__ float* at_a(const CholArgs& p, int r, int c) { return p.A + static_cast<size_t>(r) * p.n + c; }
-__device__ __forceinline__ float* at_x(const CholArgs& p, int r, int c) {
-  return p.U + static_cast<size_t>(p.n - 1 - r) * p.n + (p.n - 1 - c);
-}
+__device__ __forceinline__ float* at_a(const CholArgs& p, int r, int c) { return p.A + r * p.lda + c; }
+__device__ __forceinline__ float* at_x(const CholArgs& p, int r, int c) { return p.X + r * p.ldx + c; }
 
 // acc[i][j] = sum_k P[k][tr+i] * Q[k][tc+j]  (thread owns a 4x4 block)
 __device__ __forceinline__ void tile_product(const Tile* P, const Tile* Q, float (&acc)[4][4]) {
@@ -320,47 +346,28 @@ __device__ __forceinline__ TileOp op_phase_u(int k, int nb, int t) {
   return {kOpInverse, (k + 1 + tt / (k + 1)) * kT, (tt % (k + 1)) * kT};
 }
 
-// Four consecutive entries (r, c .. c + 3) of A or of X (X rotated into U,
-// so they lie in reverse order); c % 4 == 0.  Vector loads when p.vec.
-__device__ __forceinline__ float4 ld4_a(const CholArgs& p, int r, int c) {
+// Four consecutive entries (r, c .. c + 3) of A or of X; c % 4 == 0.  Vector
+// loads when p.vec.
+__device__ __forceinline__ float4 ld4(const CholArgs& p, bool from_x, int r, int c) {
   if (r >= p.n || c >= p.n) return make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  const float* src = p.A + static_cast<size_t>(r) * p.n + c;
+  const float* src = from_x ? at_x(p, r, c) : at_a(p, r, c);
   if (p.vec) return __ldcg(reinterpret_cast<const float4*>(src));
   return make_float4(__ldcg(src), c + 1 < p.n ? __ldcg(src + 1) : 0.0f, c + 2 < p.n ? __ldcg(src + 2) : 0.0f,
                      c + 3 < p.n ? __ldcg(src + 3) : 0.0f);
 }
-__device__ __forceinline__ float4 ld4_x(const CholArgs& p, int r, int c) {
-  if (r >= p.n || c >= p.n) return make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  const float* row = p.U + static_cast<size_t>(p.n - 1 - r) * p.n + (p.n - 1);
-  if (p.vec) {
-    const float4 v = __ldcg(reinterpret_cast<const float4*>(row - c - 3));
-    return make_float4(v.w, v.z, v.y, v.x);
-  }
-  return make_float4(__ldcg(row - c), c + 1 < p.n ? __ldcg(row - c - 1) : 0.0f,
-                     c + 2 < p.n ? __ldcg(row - c - 2) : 0.0f, c + 3 < p.n ? __ldcg(row - c - 3) : 0.0f);
-}
+__device__ __forceinline__ float4 ld4_a(const CholArgs& p, int r, int c) { return ld4(p, false, r, c); }
+__device__ __forceinline__ float4 ld4_x(const CholArgs& p, int r, int c) { return ld4(p, true, r, c); }
+
 __device__ __forceinline__ void st4(const CholArgs& p, bool to_x, int r, int c, float4 v) {
   if (r >= p.n || c >= p.n) return;
-  if (!to_x) {
-    float* dst = p.A + static_cast<size_t>(r) * p.n + c;
-    if (p.vec) {
-      *reinterpret_cast<float4*>(dst) = v;
-    } else {
-      dst[0] = v.x;
-      if (c + 1 < p.n) dst[1] = v.y;
-      if (c + 2 < p.n) dst[2] = v.z;
-      if (c + 3 < p.n) dst[3] = v.w;
-    }
+  float* dst = to_x ? at_x(p, r, c) : at_a(p, r, c);
+  if (p.vec) {
+    *reinterpret_cast<float4*>(dst) = v;
   } else {
-    float* row = p.U + static_cast<size_t>(p.n - 1 - r) * p.n + (p.n - 1);
-    if (p.vec) {
-      *reinterpret_cast<float4*>(row - c - 3) = make_float4(v.w, v.z, v.y, v.x);
-    } else {
-      row[-c] = v.x;
-      if (c + 1 < p.n) row[-c - 1] = v.y;
-      if (c + 2 < p.n) row[-c - 2] = v.z;
-      if (c + 3 < p.n) row[-c - 3] = v.w;
-    }
+    dst[0] = v.x;
+    if (c + 1 < p.n) dst[1] = v.y;
+    if (c + 2 < p.n) dst[2] = v.z;
+    if (c + 3 < p.n) dst[3] = v.w;
   }
 }
 
@@ -370,29 +377,15 @@ __device__ __forceinline__ void st4(const CholArgs& p, bool to_x, int r, int c, 
 // a load, an fp32 addition and a store.
 __device__ __forceinline__ void red4(const CholArgs& p, bool to_x, int r, int c, float4 v) {
   if (r >= p.n || c >= p.n) return;
-  if (!to_x) {
-    float* dst = p.A + static_cast<size_t>(r) * p.n + c;
-    if (p.vec) {
-      asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
-                   : "memory");
-    } else {
-      atomicAdd(dst, v.x);
-      if (c + 1 < p.n) atomicAdd(dst + 1, v.y);
-      if (c + 2 < p.n) atomicAdd(dst + 2, v.z);
-      if (c + 3 < p.n) atomicAdd(dst + 3, v.w);
-    }
+  float* dst = to_x ? at_x(p, r, c) : at_a(p, r, c);
+  if (p.vec) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+                 : "memory");
   } else {
-    float* row = p.U + static_cast<size_t>(p.n - 1 - r) * p.n + (p.n - 1);
-    if (p.vec) {
-      asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(row - c - 3), "f"(v.w), "f"(v.z), "f"(v.y),
-                   "f"(v.x)
-                   : "memory");
-    } else {
-      atomicAdd(row - c, v.x);
-      if (c + 1 < p.n) atomicAdd(row - c - 1, v.y);
-      if (c + 2 < p.n) atomicAdd(row - c - 2, v.z);
-      if (c + 3 < p.n) atomicAdd(row - c - 3, v.w);
-    }
+    atomicAdd(dst, v.x);
+    if (c + 1 < p.n) atomicAdd(dst + 1, v.y);
+    if (c + 2 < p.n) atomicAdd(dst + 2, v.z);
+    if (c + 3 < p.n) atomicAdd(dst + 3, v.w);
   }
 }
 
@@ -577,8 +570,18 @@ __global__ void __launch_bounds__(kCholThreads, 2) chol_inv_kernel(CholArgs p) {
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+constexpr int kNB = 1024;  // diagonal block of the blocked factorization
+// From this order on, 1024-wide blocks joined by tensor-core GEMMs.  Below it
+// the single cooperative kernel is faster (2.9 vs 4.4 ms at 4096: the blocked
+// form runs the same 64-wide panel chain plus the GEMM launches) and more
+// accurate (U^T U H' v = v to ~7e-7 vs ~4e-6: the tensor-core accumulation
+// of each 128-long K chunk rounds like truncation).  At 8192 the two take the
+// same time; at 11008 the blocked form is 1.15x faster, and its advantage
+// grows with n (its O(n^3) part runs on the tensor cores).
+constexpr int kBlockedMinN = 8192;
+
 struct PrepLayout {
-  size_t a, key, dead, lambda, bar, perm, total;
+  size_t a, key, dead, lambda, bar, perm, ahi, alo, bhi, blo, panel, total;
 };
 
 PrepLayout prep_layout(int n) {
@@ -597,6 +600,19 @@ PrepLayout prep_layout(int n) {
   off += 256 + align256(kMaxCholCtas * sizeof(unsigned));
   l.perm = off;
   off += align256(static_cast<size_t>(n) * sizeof(int32_t));
+  // blocked factorization (n > kNB): tf32 halves of the GEMM operands and the
+  // panel L_>K,K, each at most n x kNB
+  const size_t blk = n >= kBlockedMinN ? align256(static_cast<size_t>(n) * kNB * sizeof(float)) : 0;
+  l.ahi = off;
+  off += blk;
+  l.alo = off;
+  off += blk;
+  l.bhi = off;
+  off += blk;
+  l.blo = off;
+  off += blk;
+  l.panel = off;
+  off += blk;
   l.total = off;
   return l;
 }
@@ -616,6 +632,13 @@ int chol_grid(const DeviceInfo* info) {
 }  // namespace
 
 size_t prepare_workspace_size(int n) { return n > 0 ? prep_layout(n).total : 0; }
+
+gptq_status split_rows_tf32(const float* src, int64_t lds, int rows, int cols, int kpad, float sign, float* hi,
+                            float* lo, cudaStream_t st);
+gptq_status split_cols_tf32(const float* src, int64_t lds, int rows, int cols, int kpad, float sign, float* hi,
+                            float* lo, cudaStream_t st);
+gptq_status gemm_nt_tc(float* C, int64_t ldc, int M, int N, int kpad, const float* A_hi, const float* A_lo,
+                       const float* B_hi, const float* B_lo, cudaStream_t st);
 
 gptq_status prepare_hinv(const float* H, const double* hdiag, int n, float damp, int act_order, int32_t* perm_out,
                          uint8_t* dead_out, float* U, void* ws, size_t ws_bytes, cudaStream_t st) {
@@ -656,22 +679,73 @@ gptq_status prepare_hinv(const float* H, const double* hdiag, int n, float damp,
   if (cudaMemsetAsync(U, 0, static_cast<size_t>(n) * n * sizeof(float), st) != cudaSuccess) return GPTQ_ERR_CUDA;
   if (launch_status() != GPTQ_OK) return GPTQ_ERR_CUDA;
 
-  CholArgs ca;
-  ca.A = A;
-  ca.U = U;
-  ca.n = n;
-  ca.nblk = static_cast<int>(ceil_div(n, kT));
-  ca.fstatus = fstatus;
-  ca.bar = bar;
-  ca.abort = reinterpret_cast<int*>(bar + 2);
-  ca.smids = bar + 64;
-  ca.wait_ns = wait_limit_ns();
-  ca.vec = (n % 4 == 0) ? 1 : 0;
-  void* args[] = {&ca};
-  if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(chol_inv_kernel), dim3(grid), dim3(kCholThreads),
-                                  args, kCholSmem, st) != cudaSuccess)
-    return GPTQ_ERR_CUDA;
-  count_launch();
+  // The diagonal block [k0, k0 + kb) through the cooperative kernel; X = U
+  // (unrotated until the end).
+  auto factor_block = [&](int k0, int kb) -> gptq_status {
+    if (cudaMemsetAsync(bar, 0, 256, st) != cudaSuccess) return GPTQ_ERR_CUDA;
+    CholArgs ca;
+    ca.A = A + static_cast<int64_t>(k0) * n + k0;
+    ca.X = U + static_cast<int64_t>(k0) * n + k0;
+    ca.lda = n;
+    ca.ldx = n;
+    ca.n = kb;
+    ca.nblk = static_cast<int>(ceil_div(kb, kT));
+    ca.fstatus = fstatus;
+    ca.bar = bar;
+    ca.abort = reinterpret_cast<int*>(bar + 2);
+    ca.smids = bar + 64;
+    ca.wait_ns = wait_limit_ns();
+    ca.vec = (n % 4 == 0) ? 1 : 0;
+    void* args[] = {&ca};
+    if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(chol_inv_kernel), dim3(grid), dim3(kCholThreads),
+                                    args, kCholSmem, st) != cudaSuccess)
+      return GPTQ_ERR_CUDA;
+    count_launch();
+    return GPTQ_OK;
+  };
+  float* Ahi = reinterpret_cast<float*>(w + l.ahi);
+  float* Alo = reinterpret_cast<float*>(w + l.alo);
+  float* Bhi = reinterpret_cast<float*>(w + l.bhi);
+  float* Blo = reinterpret_cast<float*>(w + l.blo);
+  float* P = reinterpret_cast<float*>(w + l.panel);
+  const int nb_outer = n >= kBlockedMinN ? kNB : n;  // one block: the cooperative kernel alone
+  for (int k0 = 0; k0 < n; k0 += nb_outer) {
+    const int kb = std::min(nb_outer, n - k0), k1 = k0 + kb, m = n - k1;
+    const int kp = static_cast<int>(ceil_div(kb, 32)) * 32;  // padded contraction length
+    float* XK = U + static_cast<int64_t>(k0) * n;             // block row K of X (and of R)
+    float* XKK = XK + k0;
+    gptq_status s = factor_block(k0, kb);
+    if (s != GPTQ_OK) return s;
+    if (k0 > 0) {
+      // finalize: X_K,<K = X_KK R_K,<K  (R_K,<K split, then its place zeroed)
+      if ((s = split_cols_tf32(XK, n, kb, k0, kp, 1.0f, Bhi, Blo, st)) != GPTQ_OK) return s;
+      if (cudaMemset2DAsync(XK, static_cast<size_t>(n) * 4, 0, static_cast<size_t>(k0) * 4, kb, st) != cudaSuccess)
+        return GPTQ_ERR_CUDA;
+      if ((s = split_rows_tf32(XKK, n, kb, kb, kp, -1.0f, Ahi, Alo, st)) != GPTQ_OK) return s;
+      if ((s = gemm_nt_tc(XK, n, kb, k0, kp, Ahi, Alo, Bhi, Blo, st)) != GPTQ_OK) return s;
+    }
+    if (m == 0) break;
+    // panel: L_>K,K = A_>K,K X_KK^T into P [m, kp]
+    float* AIK = A + static_cast<int64_t>(k1) * n + k0;
+    if ((s = split_rows_tf32(AIK, n, m, kb, kp, -1.0f, Ahi, Alo, st)) != GPTQ_OK) return s;
+    if ((s = split_rows_tf32(XKK, n, kb, kb, kp, 1.0f, Bhi, Blo, st)) != GPTQ_OK) return s;
+    if (cudaMemsetAsync(P, 0, static_cast<size_t>(m) * kp * sizeof(float), st) != cudaSuccess) return GPTQ_ERR_CUDA;
+    if ((s = gemm_nt_tc(P, kp, m, kb, kp, Ahi, Alo, Bhi, Blo, st)) != GPTQ_OK) return s;
+    // trailing update: A_>K,>K -= P P^T
+    if ((s = split_rows_tf32(P, kp, m, kb, kp, 1.0f, Ahi, Alo, st)) != GPTQ_OK) return s;
+    if ((s = gemm_nt_tc(A + static_cast<int64_t>(k1) * n + k1, n, m, m, kp, Ahi, Alo, Ahi, Alo, st)) != GPTQ_OK)
+      return s;
+    // inverse update: R_>K,<=K -= P X_K,<=K
+    if ((s = split_cols_tf32(XK, n, kb, k1, kp, 1.0f, Bhi, Blo, st)) != GPTQ_OK) return s;
+    if ((s = gemm_nt_tc(U + static_cast<int64_t>(k1) * n, n, m, k1, kp, Ahi, Alo, Bhi, Blo, st)) != GPTQ_OK)
+      return s;
+  }
+  {
+    const int64_t count = static_cast<int64_t>(n) * n;
+    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(ceil_div(count / 2, 256), 148 * 16));
+    launch(reverse_kernel, static_cast<unsigned>(blocks), 256, 0, st, U, count);
+    if (launch_status() != GPTQ_OK) return GPTQ_ERR_CUDA;
+  }
 
   int fs = 0;
   if (cudaMemcpyAsync(&fs, fstatus, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return GPTQ_ERR_CUDA;

@@ -17,7 +17,9 @@
 // zeros in a micro-test), so U's split halves are stored transposed:
 // Ut_hi[c][k] = hi(U[k][c]).
 //
-// Kernel: persistent CTAs over 128 x 256 output tiles; a TMA producer warp
+// Kernel: persistent CTAs over 128 x 256 output tiles (each tile's K range in
+// one or more accumulation units, subtracted from W one after another); a TMA
+// producer warp
 // fills a 2-stage ring (per stage 32 columns of K: E_hi and E_lo as 128 x 32
 // boxes, Ut_hi and Ut_lo as 256 x 32 boxes), one thread issues the MMAs into a
 // double-buffered 2 x 256-column accumulator, and four epilogue warps read it
@@ -42,11 +44,21 @@ constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 constexpr size_t kSmemBytes = 1024 + size_t(kStages) * kStageBytes + 256;
 constexpr uint64_t kDrainNs = 2000000000ull;
+// K chunks (of kBK) per accumulation unit in the factorization's GEMMs: each
+// unit's product goes through tensor memory on its own and is subtracted from
+// the output in fp32 by the epilogue (one read-modify-write of the tile per
+// unit, L2-resident for consecutive units of a tile).  The tensor-core
+// accumulator rounds like truncation, so its error grows with the number of
+// MMAs it sums; 128 columns of K keep it near an fp32 product's.  The column
+// loop's updates use one unit for the whole K (<= 1024), which its parity
+// tests show to be accurate enough, and save the extra passes over W.
+constexpr int kGemmUnitChunks = 4;
 
 struct TrailParams {
   float* W;        // [M, ldw]
   int64_t ldw;
   int M, N, K;     // rows, output columns, contraction length (multiple of 32)
+  int unit_chunks; // K chunks (of kBK) accumulated in tensor memory before each subtraction
   int c0, k0;      // first output column of W (and of U), first row of U
   int tiles_m, tiles_n;
   int* status;
@@ -140,49 +152,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0, local = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++local) {
-        const int buf = local & 1;
-        const uint32_t acc_phase = static_cast<uint32_t>(local >> 1) & 1u;
-        if (!mbar_wait(acc_empty + buf, acc_phase ^ 1u, p.wait_ns) || *abort_flag) {
-          set_status(p.status, GPTQ_ERR_TIMEOUT);
-          *abort_flag = 1;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kBN);
-        for (int kc = 0; kc < kchunks; ++kc) {
-          if (!mbar_wait(full + stage, phase, p.wait_ns) || *abort_flag) {
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        // one accumulation unit per p.unit_chunks chunks of K
+        for (int u0 = 0; u0 < kchunks && ok; u0 += p.unit_chunks, ++local) {
+          const int u1 = min(u0 + p.unit_chunks, kchunks);
+          const int buf = local & 1;
+          const uint32_t acc_phase = static_cast<uint32_t>(local >> 1) & 1u;
+          if (!mbar_wait(acc_empty + buf, acc_phase ^ 1u, p.wait_ns) || *abort_flag) {
             set_status(p.status, GPTQ_ERR_TIMEOUT);
             *abort_flag = 1;
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_hi = smem_u32(ring + size_t(stage) * kStageBytes);
-          const uint32_t a_lo = a_hi + kABytes;
-          const uint32_t b_hi = a_lo + kABytes;
-          const uint32_t b_lo = b_hi + kBBytes;
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kBN);
+          for (int kc = u0; kc < u1; ++kc) {
+            if (!mbar_wait(full + stage, phase, p.wait_ns) || *abort_flag) {
+              set_status(p.status, GPTQ_ERR_TIMEOUT);
+              *abort_flag = 1;
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a_hi = smem_u32(ring + size_t(stage) * kStageBytes);
+            const uint32_t a_lo = a_hi + kABytes;
+            const uint32_t b_hi = a_lo + kABytes;
+            const uint32_t b_lo = b_hi + kBBytes;
 #pragma unroll
-          for (int kk = 0; kk < kBK / 8; ++kk) {
-            // K-major: the next 8 columns of K are 32 bytes further along
-            // each 128-byte row.
-            const uint64_t dah = smem_desc_sw128(a_hi + kk * 32, 16, 1024);
-            const uint64_t dal = smem_desc_sw128(a_lo + kk * 32, 16, 1024);
-            const uint64_t dbh = smem_desc_sw128(b_hi + kk * 32, 16, 1024);
-            const uint64_t dbl = smem_desc_sw128(b_lo + kk * 32, 16, 1024);
-            const uint32_t acc = (kc > 0 || kk > 0) ? 1u : 0u;
-            mma_tf32(d_tmem, dah, dbh, idesc, acc);
-            mma_tf32(d_tmem, dah, dbl, idesc, 1u);
-            mma_tf32(d_tmem, dal, dbh, idesc, 1u);
+            for (int kk = 0; kk < kBK / 8; ++kk) {
+              // K-major: the next 8 columns of K are 32 bytes further along
+              // each 128-byte row.
+              const uint64_t dah = smem_desc_sw128(a_hi + kk * 32, 16, 1024);
+              const uint64_t dal = smem_desc_sw128(a_lo + kk * 32, 16, 1024);
+              const uint64_t dbh = smem_desc_sw128(b_hi + kk * 32, 16, 1024);
+              const uint64_t dbl = smem_desc_sw128(b_lo + kk * 32, 16, 1024);
+              const uint32_t acc = (kc > u0 || kk > 0) ? 1u : 0u;
+              mma_tf32(d_tmem, dah, dbh, idesc, acc);
+              mma_tf32(d_tmem, dah, dbl, idesc, 1u);
+              mma_tf32(d_tmem, dal, dbh, idesc, 1u);
+            }
+            mma_commit(empty + stage);
+            if (++stage == kStages) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
-          mma_commit(empty + stage);
-          if (++stage == kStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
+          if (!ok) break;
+          mma_commit(acc_full + buf);
         }
-        if (!ok) break;
-        mma_commit(acc_full + buf);
       }
       mma_commit(drain);
       if (!mbar_wait(drain, 0u, kDrainNs)) set_status(p.status, GPTQ_ERR_TIMEOUT);
@@ -193,7 +210,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r_in_tile = quad * 32 + lane;
     const bool vec = (p.ldw % 4 == 0) && (p.c0 % 4 == 0) && (reinterpret_cast<uintptr_t>(p.W) % 16 == 0);
     int local = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++local) {
+    bool live = true;
+    for (int t = blockIdx.x; t < num_tiles && live; t += gridDim.x)
+    for (int u0 = 0; u0 < kchunks; u0 += p.unit_chunks, ++local) {
       const int tm = t / p.tiles_n, tn = t - tm * p.tiles_n;
       const int row = tm * kBM + r_in_tile;
       const int col0 = p.c0 + tn * kBN;
@@ -209,7 +228,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
+      if (!ok) {
+        live = false;
+        break;
+      }
       tc_fence_after();
       float* wrow = p.W + static_cast<int64_t>(row) * p.ldw + col0;
       for (int c = 0; c < kBN; c += 32) {
@@ -274,6 +296,54 @@ __global__ void split_transpose_tf32_kernel(const float* __restrict__ U, int n, 
   }
 }
 
+// hi[i][k] / lo[i][k] (i < rows, k < kpad, pitch kpad) = tf32 split of
+// sign * src[i][k] for k < cols, zero for cols <= k < kpad.
+__global__ void split_rows_tf32_kernel(const float* __restrict__ src, int64_t lds, int rows, int cols, int kpad,
+                                       float sign, float* __restrict__ hi, float* __restrict__ lo) {
+  const int i = blockIdx.y;
+  if (i >= rows) return;
+  for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < kpad; k += gridDim.x * blockDim.x) {
+    const float x = k < cols ? sign * src[static_cast<int64_t>(i) * lds + k] : 0.0f;
+    const float h = __uint_as_float(__float_as_uint(x) & 0xffffe000u);
+    hi[static_cast<int64_t>(i) * kpad + k] = h;
+    lo[static_cast<int64_t>(i) * kpad + k] = x - h;
+  }
+}
+
+// hi[j][k] / lo[j][k] (j < cols, k < kpad, pitch kpad) = tf32 split of
+// sign * src[k][j] for k < rows, zero beyond: the transpose, through 32 x 32
+// shared-memory tiles.
+__global__ void split_cols_tf32_kernel(const float* __restrict__ src, int64_t lds, int rows, int cols, int kpad,
+                                       float sign, float* __restrict__ hi, float* __restrict__ lo) {
+  __shared__ float t[32][33];
+  const int k0 = blockIdx.y * 32, j0 = blockIdx.x * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int k = k0 + i, j = j0 + threadIdx.x;
+    t[i][threadIdx.x] = (k < rows && j < cols) ? sign * src[static_cast<int64_t>(k) * lds + j] : 0.0f;
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int j = j0 + i, k = k0 + threadIdx.x;
+    if (j < cols && k < kpad) {
+      const float x = t[threadIdx.x][i];
+      const float h = __uint_as_float(__float_as_uint(x) & 0xffffe000u);
+      hi[static_cast<int64_t>(j) * kpad + k] = h;
+      lo[static_cast<int64_t>(j) * kpad + k] = x - h;
+    }
+  }
+}
+
+bool set_smem_attr(const DeviceInfo* info) {
+  static bool attr_set[64] = {};
+  if (!attr_set[info->device]) {
+    if (cudaFuncSetAttribute(trailing_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBytes)) != cudaSuccess)
+      return false;
+    attr_set[info->device] = true;
+  }
+  return true;
+}
+
 }  // namespace
 
 // Splits U [n, n] into transposed tf32 hi / lo halves with row pitch ldu.
@@ -305,19 +375,14 @@ gptq_status trailing_update_tc(float* W, int64_t ldw, int M, int N, int K, int c
       !make_tensor_map_2d(&m_ulo, f32, U_lo, static_cast<uint64_t>(n_u), static_cast<uint64_t>(n_u),
                           static_cast<uint64_t>(ldu) * 4, kBK, kBN, CU_TENSOR_MAP_SWIZZLE_128B))
     return GPTQ_ERR_CUDA;
-  static bool attr_set[64] = {};
-  if (!attr_set[info->device]) {
-    if (cudaFuncSetAttribute(trailing_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemBytes)) != cudaSuccess)
-      return GPTQ_ERR_CUDA;
-    attr_set[info->device] = true;
-  }
+  if (!set_smem_attr(info)) return GPTQ_ERR_CUDA;
   TrailParams p;
   p.W = W;
   p.ldw = ldw;
   p.M = M;
   p.N = N;
   p.K = K;
+  p.unit_chunks = K / kBK;  // one unit: the whole contraction
   p.c0 = c0;
   p.k0 = k0;
   p.tiles_m = static_cast<int>(ceil_div(M, kBM));
@@ -326,6 +391,63 @@ gptq_status trailing_update_tc(float* W, int64_t ldw, int M, int N, int K, int c
   p.wait_ns = wait_limit_ns();
   const int grid = std::min(info->sm_count, p.tiles_m * p.tiles_n);
   launch(trailing_tc_kernel, grid, kThreads, kSmemBytes, st, m_ehi, m_elo, m_uhi, m_ulo, p);
+  return launch_status();
+}
+
+
+gptq_status split_rows_tf32(const float* src, int64_t lds, int rows, int cols, int kpad, float sign, float* hi,
+                            float* lo, cudaStream_t st) {
+  if (rows <= 0 || kpad <= 0) return GPTQ_OK;
+  const dim3 grid(static_cast<unsigned>(std::min<int64_t>(ceil_div(kpad, 256), 8)), static_cast<unsigned>(rows));
+  launch(split_rows_tf32_kernel, grid, 256, 0, st, src, lds, rows, cols, kpad, sign, hi, lo);
+  return launch_status();
+}
+
+gptq_status split_cols_tf32(const float* src, int64_t lds, int rows, int cols, int kpad, float sign, float* hi,
+                            float* lo, cudaStream_t st) {
+  if (cols <= 0 || kpad <= 0) return GPTQ_OK;
+  const dim3 grid(static_cast<unsigned>(ceil_div(cols, 32)), static_cast<unsigned>(ceil_div(kpad, 32)));
+  launch(split_cols_tf32_kernel, grid, dim3(32, 8), 0, st, src, lds, rows, cols, kpad, sign, hi, lo);
+  return launch_status();
+}
+
+// C[M, N] -= A[M, K] B[N, K]^T (fp32-accurate), A and B given as tf32 hi / lo
+// halves, row-major with K contiguous and row pitch kpad (a multiple of 32,
+// zero-padded past K).  C has row pitch ldc; any alignment.
+gptq_status gemm_nt_tc(float* C, int64_t ldc, int M, int N, int kpad, const float* A_hi, const float* A_lo,
+                       const float* B_hi, const float* B_lo, cudaStream_t st) {
+  const DeviceInfo* info = device_info();
+  if (info == nullptr) return GPTQ_ERR_CUDA;
+  if (M <= 0 || N <= 0 || kpad <= 0) return GPTQ_OK;
+  if (kpad % kBK != 0) return GPTQ_ERR_INVALID_ARG;
+  if (!set_smem_attr(info)) return GPTQ_ERR_CUDA;
+  const CUtensorMapDataType f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  const uint64_t pitch = static_cast<uint64_t>(kpad) * 4;
+  CUtensorMap m_ahi, m_alo, m_bhi, m_blo;
+  if (!make_tensor_map_2d(&m_ahi, f32, A_hi, kpad, static_cast<uint64_t>(M), pitch, kBK, kBM,
+                          CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tensor_map_2d(&m_alo, f32, A_lo, kpad, static_cast<uint64_t>(M), pitch, kBK, kBM,
+                          CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tensor_map_2d(&m_bhi, f32, B_hi, kpad, static_cast<uint64_t>(N), pitch, kBK, kBN,
+                          CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tensor_map_2d(&m_blo, f32, B_lo, kpad, static_cast<uint64_t>(N), pitch, kBK, kBN,
+                          CU_TENSOR_MAP_SWIZZLE_128B))
+    return GPTQ_ERR_CUDA;
+  TrailParams p;
+  p.W = C;
+  p.ldw = ldc;
+  p.M = M;
+  p.N = N;
+  p.K = kpad;
+  p.unit_chunks = kGemmUnitChunks;
+  p.c0 = 0;
+  p.k0 = 0;
+  p.tiles_m = static_cast<int>(ceil_div(M, kBM));
+  p.tiles_n = static_cast<int>(ceil_div(N, kBN));
+  p.status = info->status;
+  p.wait_ns = wait_limit_ns();
+  const int grid = std::min(info->sm_count, p.tiles_m * p.tiles_n);
+  launch(trailing_tc_kernel, grid, kThreads, kSmemBytes, st, m_ahi, m_alo, m_bhi, m_blo, p);
   return launch_status();
 }
 

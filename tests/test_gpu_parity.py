@@ -164,8 +164,12 @@ def _spd_from_x(n, n_tok, seed, dead=()):
     return X, Hx
 
 
-@pytest.mark.parametrize("n,act_order", [(64, False), (200, True), (256, False), (515, True), (1024, False)])
+@pytest.mark.parametrize("n,act_order", [(64, False), (200, True), (256, False), (515, True), (1024, False),
+                                        (2600, True), (3001, False), (8200, True)])
 def test_prepare_matches_oracle(n, act_order):
+    """Below n = 8192 one cooperative factorization (3001: rows not 16-byte
+    aligned); 8200: 1024-wide diagonal blocks joined by tensor-core GEMMs, with
+    a ragged last block and act-order."""
     X, Hx = _spd_from_x(n, 4 * n, seed=n, dead=(3,))
     H32 = torch.tensor(Hx.astype(np.float32), device="cuda")
     U, perm, dead = gq.gptq_prepare_hinv(H32, 0.01, act_order)
@@ -293,6 +297,29 @@ def test_two_level_blocking_matches_oracle(name, rows, n, group, block):
     assert agree >= 0.999, agree
     assert abs(err_gpu - err_ref) <= 1e-3 * err_ref, (err_gpu, err_ref)
     np.testing.assert_allclose(npx(out["row_loss"]), ref["row_loss"], rtol=2e-2)
+
+
+def test_layer_with_blocked_factorization_matches_oracle():
+    """n = 8192: U comes from the blocked factorization (tensor-core GEMMs
+    between 1024-wide diagonal blocks).  H is formed on the host in fp64 and
+    handed, rounded to fp32, to both sides, so the check covers the factor and
+    the column loop alone; codes and output error meet the parity bar."""
+    spec = si.scaled(si.SPECS["attn4096"], rows=16, n=8192, n_tok=16384)
+    W = si.make_weights(spec, "cuda")
+    X = si.make_activations(spec, "cpu")
+    S = go.accumulate_hessian(np.zeros((spec.n, spec.n)), X.double().numpy(), 1.0)
+    H32 = ((2.0 / spec.n_tok) * S).astype(np.float32)
+    U, perm, dead = gq.gptq_prepare_hinv(torch.tensor(H32, device="cuda"), spec.damp, False)
+    out = gq.gptq_quantize_layer(W, U, spec.bits, spec.group, spec.block, dead=dead, want_deq=True)
+    torch.cuda.synchronize()
+    Wh = np64(W)
+    ref = go.gptq_layer(Wh, H=H32.astype(np.float64), bits=spec.bits, group=spec.group, damp=spec.damp,
+                        block=spec.block)
+    agree = float(np.mean(npx(out["codes"]).astype(np.int64) == ref["codes"]))
+    assert agree >= 0.999, agree
+    err_gpu = go.layer_output_error(Wh, np64(out["deq"]), S)
+    err_ref = go.layer_output_error(Wh, ref["deq"], S)
+    assert abs(err_gpu - err_ref) <= 1e-3 * err_ref, (err_gpu, err_ref)
 
 
 def test_dead_columns_and_bf16_weights():
