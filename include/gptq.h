@@ -147,7 +147,9 @@ size_t gptq_prepare_workspace_size(int32_t n);
  * one triangular inverse), which equals the upper Cholesky factor of the
  * inverse.
  *
- *   H        fp32 [n, n] symmetric, read only (the lower triangle is used).
+ *   H        fp32 [n, n] symmetric, read only (entries of either triangle are
+ *            read, so both must hold the same values, as gptq_hessian_accum
+ *            writes them).
  *   hdiag    fp64 [n] or NULL: the key for dead columns and act-order
  *            (NULL: the fp32 diagonal of H).
  *   damp     relative damping, >= 0 and finite.
