@@ -56,6 +56,27 @@ def dist_env():
     return world, rank, local
 
 
+def rank_seed(seed, rank):
+    """Each rank quantizes its own layer: a distinct seed per rank."""
+    return seed + 7919 * rank
+
+
+def max_over_ranks(value, dist, device):
+    """The slowest rank's time (every rank receives it); `dist` is None for one
+    process."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(world, rows, n, ms):
+    """Whole-job weights per second: every rank's layer over the slowest time."""
+    return world * rows * n / (ms / 1e3)
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -212,7 +233,7 @@ def run_ours(args, world, rank, local):
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
     base = si.SPECS[args.workload]
-    spec = si.scaled(base, seed=base.seed + 7919 * rank, n_tok=args.tokens or base.n_tok)
+    spec = si.scaled(base, seed=rank_seed(base.seed, rank), n_tok=args.tokens or base.n_tok)
     W, X = si.make_layer(spec, dev)
     n, rows = spec.n, spec.rows
     ng = gq.LIB.gptq_num_groups(n, spec.group)
@@ -292,16 +313,13 @@ def run_ours(args, world, rank, local):
     elapsed_ms = t_start.elapsed_time(t_end)
     stages = [[e[i].elapsed_time(e[i + 1]) for e in step_events] for i in range(nev - 1)]
     stage_ms = [statistics.mean(s) for s in stages]
-    if dist is not None:
-        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, dist, dev)
     status = gq.gptq_get_device_status()
     if status != 0:
         raise RuntimeError(f"device status after the timed region: {status}")
 
     ms_per_step = elapsed_ms / args.steps
-    value = world * rows * n / (ms_per_step / 1e3)
+    value = job_rate(world, rows, n, ms_per_step)
 
     pk, pk_src = peaks()
     flops_syrk = float(n) * (n + 1) * spec.n_tok
@@ -422,12 +440,8 @@ def run_e2e(args, spec, W, X, dev, world, dist):
         one()
     e.record(stream)
     torch.cuda.synchronize()
-    ms = s.elapsed_time(e) / args.e2e_steps
-    if dist is not None:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    return {"value": world * spec.rows * spec.n / (ms / 1e3), "unit": UNIT, "ms_per_step": ms,
+    ms = max_over_ranks(s.elapsed_time(e) / args.e2e_steps, dist, dev)
+    return {"value": job_rate(world, spec.rows, spec.n, ms), "unit": UNIT, "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
 
 
