@@ -46,18 +46,19 @@ __device__ __forceinline__ float load_w<float>(const float* p) { return *p; }
 template <>
 __device__ __forceinline__ float load_w<__nv_bfloat16>(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 
-// Wk[r, p] = dead[perm[p]] ? 0 : W[r, perm[p]]  (processing order, fp32).
+// Wk[r, p] = dead[perm[p]] ? 0 : W[r, perm[p]]  (processing order, fp32);
+// rows along blockIdx.y, so no division per element.
 template <typename T>
 __global__ void gather_weights_kernel(const T* __restrict__ W, const int32_t* __restrict__ perm,
                                       const uint8_t* __restrict__ dead, int64_t rows, int n, float* __restrict__ Wk) {
-  const int64_t total = rows * n;
-  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
-       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = e / n;
-    const int p = static_cast<int>(e - r * n);
-    const int c = perm != nullptr ? perm[p] : p;
-    const bool d = dead != nullptr && dead[c];
-    Wk[e] = d ? 0.0f : load_w<T>(W + r * n + c);
+  for (int64_t r = blockIdx.y; r < rows; r += gridDim.y) {
+    const T* src = W + r * n;
+    float* dst = Wk + r * n;
+    for (int p = blockIdx.x * blockDim.x + threadIdx.x; p < n; p += gridDim.x * blockDim.x) {
+      const int c = perm != nullptr ? perm[p] : p;
+      const bool d = dead != nullptr && dead[c];
+      dst[p] = d ? 0.0f : load_w<T>(src + c);
+    }
   }
 }
 
@@ -251,29 +252,30 @@ __global__ void group_minmax_kernel(const float* __restrict__ Wk, int64_t rows, 
   if (lane == 0) out[r] = make_float2(lo, hi);
 }
 
-// codes[r, perm[p]] = codes_p[r, p]; optional dequantized weights and g_idx.
+// codes[r, perm[p]] = codes_p[r, p] and the optional dequantized weights; rows
+// along blockIdx.y, so no division per element.
 __global__ void outputs_kernel(const uint8_t* __restrict__ codes_p, const int32_t* __restrict__ perm,
                                const float* __restrict__ scales, const uint8_t* __restrict__ zeros, int64_t rows,
-                               int n, int G, int n_groups, uint8_t* __restrict__ codes, float* __restrict__ Wq,
-                               int32_t* __restrict__ g_idx) {
-  const int64_t total = rows * n;
-  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
-       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = e / n;
-    const int p = static_cast<int>(e - r * n);
+                               int n, int G, int n_groups, uint8_t* __restrict__ codes, float* __restrict__ Wq) {
+  for (int64_t r = blockIdx.y; r < rows; r += gridDim.y)
+  for (int p = blockIdx.x * blockDim.x + threadIdx.x; p < n; p += gridDim.x * blockDim.x) {
     const int c = perm != nullptr ? perm[p] : p;
-    const uint8_t q = codes_p[e];
+    const uint8_t q = codes_p[r * n + p];
     if (codes != codes_p) codes[r * n + c] = q;
-    const int g = p / G;
     if (Wq != nullptr) {
+      const int g = p / G;
       GridParams gp{scales[r * n_groups + g], static_cast<float>(zeros[r * n_groups + g])};
       Wq[r * n + c] = grid_deq(static_cast<float>(q), gp);
     }
-    if (r == 0 && g_idx != nullptr) g_idx[c] = g;
   }
 }
 
-// Round-to-nearest: one warp per (row, group), groups of G original columns.
+// g_idx[perm[p]] = p / G: the group of each original column.
+__global__ void g_idx_kernel(const int32_t* __restrict__ perm, int n, int G, int32_t* __restrict__ g_idx) {
+  const int p = blockIdx.x * blockDim.x + threadIdx.x;
+  if (p < n) g_idx[perm != nullptr ? perm[p] : p] = p / G;
+}
+
 template <typename T>
 __global__ void rtn_kernel(const T* __restrict__ W, int64_t rows, int n, int G, int n_groups, float maxq,
                            uint8_t* __restrict__ codes, float* __restrict__ scales, uint8_t* __restrict__ zeros) {
@@ -377,7 +379,8 @@ gptq_status quantize_layer(const void* W, gptq_dtype wdt, int64_t rows, int n, c
   const int G = group > 0 ? group : n;
   const int n_groups = static_cast<int>(ceil_div(n, G));
 
-  const unsigned gg = static_cast<unsigned>(std::min<int64_t>(ceil_div(rows * n, 256), 148 * 64));
+  const dim3 gg(static_cast<unsigned>(std::min<int64_t>(ceil_div(n, 256), 64)),
+                static_cast<unsigned>(std::min<int64_t>(rows, 65535)));
   if (wdt == GPTQ_BF16)
     launch(gather_weights_kernel<__nv_bfloat16>, gg, 256, 0, st, static_cast<const __nv_bfloat16*>(W), perm, dead, rows,
                                                              n, Wk);
@@ -450,7 +453,13 @@ gptq_status quantize_layer(const void* W, gptq_dtype wdt, int64_t rows, int n, c
   }
   if (launch_status() != GPTQ_OK) return GPTQ_ERR_CUDA;
   if (codes_p != codes || Wq_out != nullptr || g_idx != nullptr) {
-    launch(outputs_kernel, gg, 256, 0, st, codes_p, perm, scales, zeros, rows, n, G, n_groups, codes, Wq_out, g_idx);
+    if (codes_p != codes || Wq_out != nullptr) {
+      const dim3 og(static_cast<unsigned>(std::min<int64_t>(ceil_div(n, 256), 64)),
+                    static_cast<unsigned>(std::min<int64_t>(rows, 65535)));
+      launch(outputs_kernel, og, 256, 0, st, codes_p, perm, scales, zeros, rows, n, G, n_groups, codes, Wq_out);
+    }
+    if (g_idx != nullptr)
+      launch(g_idx_kernel, static_cast<unsigned>(ceil_div(n, 256)), 256, 0, st, perm, n, G, g_idx);
     if (launch_status() != GPTQ_OK) return GPTQ_ERR_CUDA;
   }
   return GPTQ_OK;
