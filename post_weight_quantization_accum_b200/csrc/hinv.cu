@@ -414,13 +414,32 @@ struct Staged {
 
 __device__ __forceinline__ bool q_natural(const TileOp& op) { return op.kind == kOpFinalize || op.kind == kOpInverse; }
 
-__device__ __forceinline__ void fetch_op(const CholArgs& p, const TileOp& op, int k0, Staged& st) {
+// The first operand of an operation: A_ik / L_ik (row block i of panel k) for
+// trsm, update and inverse, Linv_kk for finalize.  Consecutive operations
+// with the same key share it, so it is loaded and staged once.
+__device__ __forceinline__ int p_key(const TileOp& op) { return op.kind == kOpFinalize ? -2 : op.i0; }
+
+__device__ __forceinline__ void fetch_op(const CholArgs& p, const TileOp& op, int k0, Staged& st, bool need_p) {
 #pragma unroll
   for (int g = 0; g < 4; ++g) {
     int a, b4, an, bn4;
     slot_t(g, a, b4);
     slot_n(g, an, bn4);
     const int b = 4 * b4;
+    if (!need_p) {  // the second operand only (as in the cases below)
+      switch (op.kind) {
+        case kOpTrsm:
+          st.q[g] = ld4_x(p, k0 + a, k0 + b);
+          break;
+        case kOpUpdate:
+          st.q[g] = ld4_a(p, op.j0 + a, k0 + b);
+          break;
+        default:
+          st.q[g] = ld4_x(p, k0 + an, op.j0 + 4 * bn4);
+          break;
+      }
+      continue;
+    }
     switch (op.kind) {
       case kOpTrsm:      // A_ik * Linv_kk^T
         st.p[g] = ld4_a(p, op.i0 + a, k0 + b);
@@ -444,17 +463,19 @@ __device__ __forceinline__ void fetch_op(const CholArgs& p, const TileOp& op, in
 
 // P is always used as P[r][k]; Q as Q[c][k] (transposed load) for the
 // Cholesky operations and as Q[k][c] (natural load) for the inverse ones.
-__device__ __forceinline__ void commit_op(const TileOp& op, const Staged& st, Tile* sp, Tile* sq) {
+__device__ __forceinline__ void commit_op(const TileOp& op, const Staged& st, Tile* sp, Tile* sq, bool write_p) {
   const bool qn = q_natural(op);
 #pragma unroll
   for (int g = 0; g < 4; ++g) {
     int a, b4;
     slot_t(g, a, b4);
     const int b = 4 * b4;
-    sp[b + 0][a] = st.p[g].x;
-    sp[b + 1][a] = st.p[g].y;
-    sp[b + 2][a] = st.p[g].z;
-    sp[b + 3][a] = st.p[g].w;
+    if (write_p) {
+      sp[b + 0][a] = st.p[g].x;
+      sp[b + 1][a] = st.p[g].y;
+      sp[b + 2][a] = st.p[g].z;
+      sp[b + 3][a] = st.p[g].w;
+    }
     if (qn) {
       int an, bn4;
       slot_n(g, an, bn4);
@@ -485,33 +506,44 @@ __device__ __forceinline__ void finish_op(const CholArgs& p, const TileOp& op, i
   }
 }
 
-// Runs the tile operations t0, t0 + step, ... of one phase.  The operands of
-// the next operation are loaded into registers while the current one is
-// multiplied, so L2 latency overlaps the FMAs.
+// Runs the tile operations [lo, hi) of one phase.  Operations are numbered
+// row block by row block, so consecutive ones mostly share their first
+// operand, which then stays in shared memory.  The operands of the next
+// operation are loaded into registers while the current one is multiplied,
+// so L2 latency overlaps the FMAs.
 template <bool kPhaseU>
-__device__ void run_phase(const CholArgs& p, int k, int t0, int step, int total, Tile* s0, Tile* s1) {
-  if (t0 >= total) return;
+__device__ void run_phase(const CholArgs& p, int k, int lo, int hi, Tile* s0, Tile* s1) {
+  if (lo >= hi) return;
   const int nb = p.nblk, k0 = k * kT;
   Staged st;
-  TileOp cur = kPhaseU ? op_phase_u(k, nb, t0) : op_phase_t(k, nb, t0);
-  fetch_op(p, cur, k0, st);
-  for (int t = t0; t < total; t += step) {
-    commit_op(cur, st, s0, s1);
+  TileOp cur = kPhaseU ? op_phase_u(k, nb, lo) : op_phase_t(k, nb, lo);
+  fetch_op(p, cur, k0, st, true);
+  bool write_p = true;
+  for (int t = lo; t < hi; ++t) {
+    commit_op(cur, st, s0, s1, write_p);
     __syncthreads();
-    const int tn = t + step;
     TileOp nxt = cur;
-    if (tn < total) {
-      nxt = kPhaseU ? op_phase_u(k, nb, tn) : op_phase_t(k, nb, tn);
-      fetch_op(p, nxt, k0, st);
+    bool next_p = false;
+    if (t + 1 < hi) {
+      nxt = kPhaseU ? op_phase_u(k, nb, t + 1) : op_phase_t(k, nb, t + 1);
+      next_p = p_key(nxt) != p_key(cur);
+      fetch_op(p, nxt, k0, st, next_p);
     }
     float acc[4][4];
     tile_product(s0, s1, acc);
     finish_op(p, cur, k0, acc);
     __syncthreads();
     cur = nxt;
+    write_p = next_p;
   }
   __threadfence();  // this CTA's reductions are performed before its later reads
   __syncthreads();
+}
+
+// [lo, hi) of `total` operations for worker w of `workers` (contiguous, equal shares)
+__device__ __forceinline__ void share(int total, int w, int workers, int& lo, int& hi) {
+  lo = static_cast<int>((static_cast<int64_t>(total) * w) / workers);
+  hi = static_cast<int>((static_cast<int64_t>(total) * (w + 1)) / workers);
 }
 
 __device__ __forceinline__ unsigned sm_id() {
@@ -548,7 +580,11 @@ __global__ void __launch_bounds__(kCholThreads, 2) chol_inv_kernel(CholArgs p) {
   const int W = PT - 1;                                    // workers besides CTA 0
   for (int k = 0; k < nb; ++k) {
     // phase T(k): trsm of panel k and row k of the inverse
-    if (!idle) run_phase<false>(p, k, pidx, PT, nb - 1, s0, s1);
+    if (!idle) {
+      int lo, hi;
+      share(nb - 1, pidx, PT, lo, hi);
+      run_phase<false>(p, k, lo, hi, s0, s1);
+    }
     if (!grid_sync(p)) return;
     // phase U(k): CTA 0 updates tile (k+1, k+1) and then factors it; the
     // other CTAs share the remaining updates, so the factorization is the only
@@ -557,11 +593,13 @@ __global__ void __launch_bounds__(kCholThreads, 2) chol_inv_kernel(CholArgs p) {
     const int m = nb - k - 1;
     const int total = m * (m + 1) / 2 + m * (k + 1);
     if (W == 0) {
-      if (b == 0) run_phase<true>(p, k, 0, 1, total, s0, s1);
+      if (b == 0) run_phase<true>(p, k, 0, total, s0, s1);
     } else if (b == 0) {
-      run_phase<true>(p, k, 0, total, total, s0, s1);
-    } else if (!idle) {
-      run_phase<true>(p, k, pidx, W, total, s0, s1);
+      run_phase<true>(p, k, 0, total > 0 ? 1 : 0, s0, s1);
+    } else if (!idle && total > 1) {
+      int lo, hi;
+      share(total - 1, pidx - 1, W, lo, hi);
+      run_phase<true>(p, k, 1 + lo, 1 + hi, s0, s1);
     }
     if (b == 0 && m > 0) factor_diag(p, k + 1, s0, s1, s2);
     if (!grid_sync(p)) return;
