@@ -9,7 +9,7 @@ Every function follows the method as the source pages state it (citations are
 in each docstring) with NumPy doing the dense linear algebra.  No blocking,
 fusion or reordering is added beyond what the pages describe: the one blocked
 structure (lazy 128-column blocks with a global trailing update) is the pages'
-own.
+own.  GPTQ-2D (two-sided rounding) lives in ``oracle.gptq2d_oracle``.
 """
 from .gptq_oracle import (  # noqa: F401
     hessian,
@@ -31,3 +31,4 @@ from .gptq_oracle import (  # noqa: F401
     unpack_codes,
     packed_words_per_row,
 )
+from . import gptq2d_oracle  # noqa: F401,E402
