@@ -44,6 +44,7 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-gptq2d", action="store_true", help="skip the GPTQ-2D measurement")
     ap.add_argument("--cpu-tokens", type=int, default=8192, help="oracle sample: tokens for H")
     ap.add_argument("--cpu-rows", type=int, default=32, help="oracle sample: rows through the column loop")
     return ap.parse_args()
@@ -352,6 +353,8 @@ def run_ours(args, world, rank, local):
     if sampler:
         result["clocks"] = sampler.summary()
     result["packed_matvec"] = measure_matvec(gq, packed, out, spec, dev, pk)
+    if not args.no_gptq2d:
+        result["gptq2d"] = measure_gptq2d(gq, dev, result.get("clocks"))
 
     if not args.no_e2e:
         result["e2e"] = run_e2e(args, spec, W, X, dev, world, dist)
@@ -403,6 +406,58 @@ def measure_matvec(gq, packed, out, spec, dev, pk, copies=16, reps=64):
     return {"kernel": "dequant_matvec_kernel", "batch": 1, "us_per_call": us,
             "algorithmic_bytes": nbytes, "achieved_gbs": gbs, "peak_gbs": pk["hbm_gbs"],
             "frac": gbs / pk["hbm_gbs"], "bf16_equivalent_us_at_peak": rows * n * 2 / pk["hbm_gbs"] / 1e3}
+
+
+def measure_gptq2d(gq, dev, clocks, m=4096, n=4096, tokens=8192, reps=5):
+    """GPTQ-2D (two-sided rounding) on a 4096 x 4096 matrix, outside the timed
+    step: W ~ N(0, 0.02), a signed 4-bit grid (scale 0.005, codes clamped to
+    [-8, 7]); HL and HR are the Grams of `tokens` N(0, 1) tokens, built and
+    factored by the library (damp 0.01) before timing.  Per-call time over
+    `reps` calls after 3 warm-up calls, CUDA events on the launching stream.
+    Every call streams ~0.5 GB of W, factors and scratch (more than L2).
+    Algorithmic work: sum over entries of (i + 1) multiply-adds for the value
+    and (n - j) for the feedback row, i.e. m n (m + n) flops; the kernels are
+    fp32 FMA on the CUDA cores, so the peak is SMs x 128 lanes x 2 x clock."""
+    import torch
+
+    g = torch.Generator(device=dev).manual_seed(2)
+    U = []
+    for k in (m, n):
+        X = torch.randn((tokens, k), generator=g, device=dev).to(torch.bfloat16)
+        H = torch.zeros((k, k), dtype=torch.float32, device=dev)
+        gq.gptq_hessian_accum(H, X, 2.0 / tokens)
+        U.append(gq.gptq2d_factor(H, damp=0.01))
+        del X, H
+    W = 0.02 * torch.randn((m, n), generator=g, device=dev)
+    codes = torch.empty((m, n), dtype=torch.int32, device=dev)
+    E = torch.empty((m, n), dtype=torch.float32, device=dev)
+    ws = gq.workspace(gq.LIB.gptq2d_workspace_size(m, n), dev)
+    for _ in range(3):
+        gq.gptq2d_round(W, U[0], U[1], 0.005, -8, 7, codes=codes, E=E, ws=ws)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    launches0 = gq.gptq_kernel_launches()
+    s.record(stream)
+    for _ in range(reps):
+        gq.gptq2d_round(W, U[0], U[1], 0.005, -8, 7, codes=codes, E=E, ws=ws)
+    e.record(stream)
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / reps
+    flops = float(m) * n * (m + n)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    mhz = float((clocks or {}).get("sm_max_mhz") or 1965.0)
+    peak = sms * 128 * 2 * mhz * 1e6 / 1e12
+    achieved = flops / (ms * 1e-3) / 1e12
+    return {"workload": f"W {m}x{n} fp32 N(0, 0.02); HL, HR Grams of {tokens} N(0,1) tokens, damp 0.01; "
+                        "scale 0.005, codes in [-8, 7]",
+            "kernels": "round2d_tile_kernel + push2d_kernel per tile wavefront",
+            "ms_per_call": ms, "launches_per_call": (gq.gptq_kernel_launches() - launches0) / reps,
+            "weights_per_s": m * n / (ms * 1e-3),
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "algorithmic_flops": flops,
+                         "peak_source": f"fp32 FMA: {sms} SMs x 128 lanes x 2 flops x {mhz:.0f} MHz"}}
 
 
 def run_e2e(args, spec, W, X, dev, world, dist):

@@ -24,7 +24,9 @@
  *                           "Tradeoffs": deployment reads packed weights).
  *
  * plus gptq_quantize_rtn, the round-to-nearest baseline on the same grid
- * (knowledge note, "Common Confusions").
+ * (knowledge note, "Common Confusions"), gptq_dequant_matvec (inference with
+ * the packed weights) and gptq2d_round (GPTQ-2D, the two-sided task of the
+ * GPTQ-2D abstract on the "Daily Papers" page).
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -306,6 +308,52 @@ gptq_status gptq_dequant_matvec(const uint32_t* packed, const float* scales, con
                                 const int32_t* g_idx, int64_t rows, int32_t n, int32_t bits, int32_t group,
                                 const void* x, gptq_dtype xdt, int32_t batch, float* y, void* ws,
                                 size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* 6. GPTQ-2D: two-sided rounding                                            */
+/* ------------------------------------------------------------------------ */
+
+/* Bytes of workspace gptq2d_round needs for an m x n matrix (0 for sizes it
+ * rejects). */
+size_t gptq2d_workspace_size(int64_t m, int64_t n);
+
+/* Rounds W [m, n] to scale * integers under ||A (W - Q) B||_F^2, where only
+ * the Grams HL = A^T A and HR = B B^T enter, through their upper inverse
+ * factors:
+ *   UL  fp32 [m, m], UL^T UL = HL^-1, upper (entries below the diagonal are
+ *       never read), e.g. gptq_prepare_hinv(HL, NULL, m, 0, 0, ...);
+ *   UR  fp32 [n, n], UR^T UR = HR^-1, upper, likewise.
+ *
+ * Source: the GPTQ-2D abstract on the "Daily Papers" page.  The
+ * one-dimensional algorithm (fixed order, each rounding error fed forward
+ * through a triangular matrix) applied to vec(W) under the Kronecker Gram
+ * HL kron HR, computed anti-diagonal by anti-diagonal in cubic time: entry
+ * (i, j) is rounded at
+ *     v = W[i, j] - sum_{i' <= i} UL[i', i] * (E UR)[i', j]
+ * (E: the scaled errors of the entries already rounded, all of which lie
+ * above and to the left), q = rint(v / scale) (IEEE fp32 division, round half
+ * to even), clamped to [qmin, qmax] when clamp == 1, and its scaled error is
+ * e = (v - scale * q) / (UL[i, i] * UR[j, j]).  With HL = I this is the
+ * one-sided GPTQ column loop on every row with Hessian HR.
+ *
+ *   W       [m, n] fp32 or bf16 (wdt), row-major
+ *   scale   grid step, finite and > 0
+ *   clamp   0 (unbounded integers) or 1 (clamp to [qmin, qmax],
+ *           -2^24 <= qmin <= qmax <= 2^24)
+ *   codes   int32 [m, n] out: the integers q (Q = scale * codes)
+ *   E       fp32 [m, n] out, the scaled errors e, or NULL.  They satisfy
+ *           W - Q = UL^T E UR and tr(HL (W - Q) HR (W - Q)^T) = sum e^2.
+ *   ws      gptq2d_workspace_size(m, n) bytes, 256-byte aligned
+ * Accumulates in fp32 on the CUDA cores; about 2 * (m + n) / 64 kernel
+ * launches.  Asynchronous on `stream`.  Codes for non-finite inputs are
+ * unspecified.
+ * Errors: GPTQ_ERR_INVALID_ARG (negative sizes or sizes above 4,194,304, a bad
+ * dtype, scale or clamp range, NULL or misaligned pointers, small workspace),
+ * before any launch; GPTQ_ERR_CUDA. */
+gptq_status gptq2d_round(const void* W, gptq_dtype wdt, int64_t m, int64_t n,
+                         const float* UL, const float* UR, float scale, int32_t clamp,
+                         int32_t qmin, int32_t qmax, int32_t* codes, float* E,
+                         void* ws, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }

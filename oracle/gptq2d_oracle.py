@@ -74,13 +74,17 @@ def round_entries(v, scale, qmin=None, qmax=None):
     return q, scale * q
 
 
-def gptq2d(W, UL, UR, scale=1.0, qmin=None, qmax=None):
+def gptq2d(W, UL, UR, scale=1.0, qmin=None, qmax=None, forced=None):
     """Two-sided GPTQ, anti-diagonal by anti-diagonal (cubic form).
 
     W: [m, n]; UL: [m, m] and UR: [n, n] upper factors of HL^-1 and HR^-1.
     Returns (codes, deq, E, decision): the integer codes, scale * codes, the
     scaled errors e_ij = (wt_ij - scale * q_ij) / (UL_ii * UR_jj), and the
     values wt_ij the entries had when they were rounded.
+
+    ``forced`` (an [m, n] array of integers) replays given codes instead of
+    rounding: the feedback then follows those codes, and ``decision`` holds the
+    values at which another implementation that chose them had to decide.
     """
     W = np.asarray(W, dtype=np.float64)
     UL = np.asarray(UL, dtype=np.float64)
@@ -101,6 +105,9 @@ def gptq2d(W, UL, UR, scale=1.0, qmin=None, qmax=None):
         # current values: W[i, j] - sum_{i'} UL[i', i] * M[i', j]
         wt = W[ii, jj] - np.einsum("ki,ki->i", UL[:, ii], M[:, jj])
         q, dq = round_entries(wt, scale, qmin, qmax)
+        if forced is not None:
+            q = np.asarray(forced, dtype=np.float64)[ii, jj]
+            dq = scale * q
         e = (wt - dq) / (UL[ii, ii] * UR[jj, jj])
         codes[ii, jj] = q
         deq[ii, jj] = dq

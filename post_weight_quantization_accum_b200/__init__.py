@@ -3,7 +3,8 @@
 The functions below carry the names of the C entry points in include/gptq.h
 and only marshal arguments: torch supplies device memory and the current CUDA
 stream, the library's kernels do all of the work.  ``quantize_layer`` chains the
-four calls for one linear layer (the usual entry point for a user).
+four calls for one linear layer (the usual entry point for a user);
+``gptq2d_round`` is the two-sided rounding of the GPTQ-2D abstract.
 """
 import ctypes
 
@@ -19,6 +20,8 @@ __all__ = [
     "gptq_quantize_rtn",
     "gptq_pack",
     "gptq_dequant_matvec",
+    "gptq2d_round",
+    "gptq2d_factor",
     "gptq_get_device_status",
     "gptq_set_wait_limit_ns",
     "gptq_kernel_launches",
@@ -165,6 +168,37 @@ def gptq_dequant_matvec(packed, scales, zeros, n, bits, group, x, g_idx=None, y=
                                                          n, bits, group, _ptr(x2), xdt, batch, _ptr(y), wp, wb,
                                                          _stream(stream)))
     return y[0] if squeeze else y
+
+
+def gptq2d_factor(H, damp=0.0, ws=None, stream=None):
+    """Upper U with U^T U = (H + damp * mean(diag H) I)^-1 for a symmetric
+    positive definite Gram H (fp32 [k, k]): gptq_prepare_hinv without
+    reordering (damp 0: the Gram as given)."""
+    U, _, _ = gptq_prepare_hinv(H, damp, False, ws=ws, stream=stream)
+    return U
+
+
+def gptq2d_round(W, UL, UR, scale=1.0, qmin=None, qmax=None, want_E=True, codes=None, E=None, ws=None,
+                 stream=None):
+    """Two-sided GPTQ (GPTQ-2D): round W [m, n] (fp32 or bf16) to scale * integers
+    under tr(HL D HR D^T), given the upper factors UL (UL^T UL = HL^-1) and UR
+    (UR^T UR = HR^-1).  Clamps the integers to [qmin, qmax] when both are given.
+    Returns dict(codes=int32 [m, n], E=fp32 [m, n] scaled errors or None)."""
+    m, n = W.shape
+    dev = W.device
+    if (qmin is None) != (qmax is None):
+        raise ValueError("give both qmin and qmax, or neither")
+    clamp = 0 if qmin is None else 1
+    codes = codes if codes is not None else torch.empty((m, n), dtype=torch.int32, device=dev)
+    if want_E and E is None:
+        E = torch.empty((m, n), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = workspace(LIB.gptq2d_workspace_size(m, n), dev)
+    wp, wbytes = _ws_ptr(ws)
+    check("gptq2d_round",
+          LIB.gptq2d_round(_ptr(W), _dtype_code(W), m, n, _ptr(UL), _ptr(UR), ctypes.c_float(scale), clamp,
+                           int(qmin or 0), int(qmax or 0), _ptr(codes), _ptr(E), wp, wbytes, _stream(stream)))
+    return {"codes": codes, "E": E}
 
 
 def _hessian_from_host(H, X, hdiag, stream, chunk_tokens):

@@ -50,6 +50,10 @@ _SIGS = {
     "gptq_dequant_matvec": (ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
                                            ctypes.c_int32, _P, ctypes.c_int, ctypes.c_int32, _P, _P,
                                            ctypes.c_size_t, _P]),
+    "gptq2d_workspace_size": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64]),
+    "gptq2d_round": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int64, ctypes.c_int64, _P, _P, ctypes.c_float,
+                                    ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _P, _P, _P, ctypes.c_size_t,
+                                    _P]),
 }
 
 

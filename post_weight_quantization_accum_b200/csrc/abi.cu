@@ -1,5 +1,5 @@
 // C ABI of the library: argument validation, per-device state and dispatch to
-// the kernels in hessian.cu, hinv.cu, quantize.cu, pack.cu and matvec.cu.  Nothing here
+// the kernels in hessian.cu, hinv.cu, quantize.cu, pack.cu, matvec.cu and round2d.cu.  Nothing here
 // allocates device memory; every scratch byte comes from the caller.
 #include <atomic>
 #include <cmath>
@@ -28,6 +28,9 @@ size_t matvec_workspace_size(int n, int batch, int xdt_bf16);
 gptq_status dequant_matvec(const uint32_t* packed, const float* scales, const uint8_t* zeros, const int32_t* g_idx,
                            int64_t rows, int n, int bits, int group, const void* x, int xdt_bf16, int batch, float* y,
                            void* ws, cudaStream_t st);
+size_t round2d_workspace_size(int64_t m, int64_t n);
+gptq_status round2d(const void* W, int w_bf16, int64_t m, int64_t n, const float* UL, const float* UR, float scale,
+                    int clamp, int qmin, int qmax, int32_t* codes, float* E, void* ws, cudaStream_t st);
 
 // Status words of each device: [0] failures of asynchronous kernels (bounded
 // waits), [1] the factorization status of gptq_prepare_hinv.
@@ -243,6 +246,38 @@ gptq_status gptq_dequant_matvec(const uint32_t* packed, const float* scales, con
   if (need > 0 && (ws == nullptr || !aligned(ws, 256) || ws_bytes < need)) return GPTQ_ERR_INVALID_ARG;
   return dequant_matvec(packed, scales, zeros, g_idx, rows, n, bits, group, x, xdt == GPTQ_BF16 ? 1 : 0, batch, y, ws,
                         as_stream(stream));
+}
+
+}  // extern "C"
+
+namespace {
+// The push kernel's grid spans max(tiles) - 1 target tiles along y (<= 65535).
+constexpr int64_t kMax2dDim = 65536LL * 64;
+constexpr int32_t kMax2dCode = 1 << 24;  // codes stay exact in fp32
+}  // namespace
+
+extern "C" {
+
+size_t gptq2d_workspace_size(int64_t m, int64_t n) {
+  if (m < 0 || n < 0 || m > kMax2dDim || n > kMax2dDim) return 0;
+  return round2d_workspace_size(m, n);
+}
+
+gptq_status gptq2d_round(const void* W, gptq_dtype wdt, int64_t m, int64_t n, const float* UL, const float* UR,
+                         float scale, int32_t clamp, int32_t qmin, int32_t qmax, int32_t* codes, float* E, void* ws,
+                         size_t ws_bytes, void* stream) {
+  if (m < 0 || n < 0 || m > kMax2dDim || n > kMax2dDim || (wdt != GPTQ_F32 && wdt != GPTQ_BF16) ||
+      !(scale > 0.f) || !std::isfinite(scale) || (clamp != 0 && clamp != 1))
+    return GPTQ_ERR_INVALID_ARG;
+  if (clamp == 1 && (qmin > qmax || qmin < -kMax2dCode || qmax > kMax2dCode)) return GPTQ_ERR_INVALID_ARG;
+  if (m == 0 || n == 0) return GPTQ_OK;
+  if (W == nullptr || UL == nullptr || UR == nullptr || codes == nullptr || !aligned(W, wdt == GPTQ_BF16 ? 2 : 4) ||
+      !aligned(UL, 4) || !aligned(UR, 4) || !aligned(codes, 4) || (E != nullptr && !aligned(E, 4)))
+    return GPTQ_ERR_INVALID_ARG;
+  const size_t need = round2d_workspace_size(m, n);
+  if (ws == nullptr || !aligned(ws, 256) || ws_bytes < need) return GPTQ_ERR_INVALID_ARG;
+  return round2d(W, wdt == GPTQ_BF16 ? 1 : 0, m, n, UL, UR, scale, clamp, qmin, qmax, codes, E, ws,
+                 as_stream(stream));
 }
 
 }  // extern "C"

@@ -14,7 +14,7 @@ LIB = os.path.join(ROOT, "post_weight_quantization_accum_b200", "libgptq_b200.so
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(gptq_\w+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(gptq\w*)\s*\(", text)))
 
 
 @pytest.fixture(scope="module")
@@ -27,7 +27,8 @@ def lib():
 
 def test_header_declares_the_four_calls():
     names = declared_functions()
-    for n in ("gptq_hessian_accum", "gptq_prepare_hinv", "gptq_quantize_layer", "gptq_pack"):
+    for n in ("gptq_hessian_accum", "gptq_prepare_hinv", "gptq_quantize_layer", "gptq_pack", "gptq_dequant_matvec",
+              "gptq2d_round", "gptq2d_workspace_size"):
         assert n in names
 
 
@@ -74,3 +75,33 @@ def test_invalid_arguments_rejected_before_any_launch(lib):
     p.argtypes = [P, P, ctypes.c_int32, ctypes.c_float, ctypes.c_int32, P, P, P, P, ctypes.c_size_t, P]
     assert p(fake, None, 64, -0.1, 0, None, None, fake, fake, 1 << 30, None) == 1
     assert p(fake, None, 64, 0.01, 1, None, None, fake, fake, 1 << 30, None) == 1  # act-order needs perm
+
+
+def test_gptq2d_arguments_rejected_before_any_launch(lib):
+    P = ctypes.c_void_p
+    ws = lib.gptq2d_workspace_size
+    ws.restype = ctypes.c_size_t
+    ws.argtypes = [ctypes.c_int64, ctypes.c_int64]
+    assert ws(64, 64) == 3 * 64 * 64 * 4
+    assert ws(3, 5) == 3 * 256
+    assert ws(-1, 5) == 0
+    f = lib.gptq2d_round
+    f.argtypes = [P, ctypes.c_int, ctypes.c_int64, ctypes.c_int64, P, P, ctypes.c_float, ctypes.c_int32,
+                  ctypes.c_int32, ctypes.c_int32, P, P, P, ctypes.c_size_t, P]
+    fake = P(256)
+    big = 1 << 30
+    assert f(fake, 0, -1, 8, fake, fake, 1.0, 0, 0, 0, fake, None, fake, big, None) == 1   # negative size
+    assert f(fake, 0, 8, 8, fake, fake, 0.0, 0, 0, 0, fake, None, fake, big, None) == 1    # scale 0
+    assert f(fake, 0, 8, 8, fake, fake, float("nan"), 0, 0, 0, fake, None, fake, big, None) == 1
+    assert f(fake, 0, 8, 8, fake, fake, 1.0, 2, 0, 0, fake, None, fake, big, None) == 1     # clamp flag
+    assert f(fake, 0, 8, 8, fake, fake, 1.0, 1, 3, -3, fake, None, fake, big, None) == 1    # qmin > qmax
+    assert f(fake, 0, 8, 8, fake, fake, 1.0, 1, -(1 << 25), 0, fake, None, fake, big, None) == 1
+    assert f(fake, 3, 8, 8, fake, fake, 1.0, 0, 0, 0, fake, None, fake, big, None) == 1     # dtype
+    assert f(None, 0, 8, 8, fake, fake, 1.0, 0, 0, 0, fake, None, fake, big, None) == 1     # W NULL
+    assert f(fake, 0, 8, 8, fake, None, 1.0, 0, 0, 0, fake, None, fake, big, None) == 1     # UR NULL
+    assert f(P(258), 0, 8, 8, fake, fake, 1.0, 0, 0, 0, fake, None, fake, big, None) == 1   # fp32 W alignment
+    assert f(fake, 0, 8, 8, fake, fake, 1.0, 0, 0, 0, fake, None, fake, 100, None) == 1     # small workspace
+    assert f(fake, 0, 8, 8, fake, fake, 1.0, 0, 0, 0, fake, None, P(384 + 64), big, None) == 1  # ws alignment
+    assert f(fake, 0, 0, 8, fake, fake, 1.0, 0, 0, 0, fake, None, None, 0, None) == 0       # empty: no-op
+    assert f(fake, 0, (1 << 22) + 1, 1, fake, fake, 1.0, 0, 0, 0, fake, None, fake, big, None) == 1
+

@@ -311,3 +311,23 @@ def test_empty_and_invalid():
         g2.gptq2d(np.zeros((2, 3)), np.eye(3), np.eye(3))
     with pytest.raises(ValueError):
         g2.gptq2d(np.zeros((2, 2)), np.eye(2), np.eye(2), scale=0.0)
+
+
+def test_replaying_own_codes_is_the_identity():
+    rng = np.random.default_rng(1300)
+    m, n = 17, 23
+    HL, HR = _random_spd(rng, m), _random_spd(rng, n)
+    W = rng.standard_normal((m, n))
+    res = g2.gptq2d_from_grams(W, HL, HR, 0.3, -3, 2)
+    c, dq, E, dec = g2.gptq2d(W, res["UL"], res["UR"], 0.3, -3, 2, forced=res["codes"])
+    assert np.array_equal(c, res["codes"])
+    assert np.array_equal(E, res["E"]) and np.array_equal(dec, res["decision"])
+    # replaying a flipped code changes only the entries below and to the right
+    F = res["codes"].copy()
+    F[5, 7] += 1
+    c2, _, E2, dec2 = g2.gptq2d(W, res["UL"], res["UR"], 0.3, forced=F)
+    changed = np.argwhere(~np.isclose(dec2, res["decision"], rtol=0, atol=1e-13))
+    assert len(changed) > 0
+    assert np.all((changed[:, 0] >= 5) & (changed[:, 1] >= 7))
+    assert np.array_equal(dec2[5, 7], res["decision"][5, 7])
+
