@@ -354,7 +354,8 @@ def run_ours(args, world, rank, local):
         result["clocks"] = sampler.summary()
     result["packed_matvec"] = measure_matvec(gq, packed, out, spec, dev, pk)
     if not args.no_gptq2d:
-        result["gptq2d"] = measure_gptq2d(gq, dev, result.get("clocks"))
+        cpu_rows = 64 if (world == 1 and rank == 0 and not args.no_cpu_baseline) else 0
+        result["gptq2d"] = measure_gptq2d(gq, dev, result.get("clocks"), cpu_rows=cpu_rows)
 
     if not args.no_e2e:
         result["e2e"] = run_e2e(args, spec, W, X, dev, world, dist)
@@ -408,7 +409,7 @@ def measure_matvec(gq, packed, out, spec, dev, pk, copies=16, reps=64):
             "frac": gbs / pk["hbm_gbs"], "bf16_equivalent_us_at_peak": rows * n * 2 / pk["hbm_gbs"] / 1e3}
 
 
-def measure_gptq2d(gq, dev, clocks, m=4096, n=4096, tokens=8192, reps=5):
+def measure_gptq2d(gq, dev, clocks, m=4096, n=4096, tokens=8192, reps=5, cpu_rows=0):
     """GPTQ-2D (two-sided rounding) on a 4096 x 4096 matrix, outside the timed
     step: W ~ N(0, 0.02), a signed 4-bit grid (scale 0.005, codes clamped to
     [-8, 7]); HL and HR are the Grams of `tokens` N(0, 1) tokens, built and
@@ -417,7 +418,11 @@ def measure_gptq2d(gq, dev, clocks, m=4096, n=4096, tokens=8192, reps=5):
     Every call streams ~0.5 GB of W, factors and scratch (more than L2).
     Algorithmic work: sum over entries of (i + 1) multiply-adds for the value
     and (n - j) for the feedback row, i.e. m n (m + n) flops; the kernels are
-    fp32 FMA on the CUDA cores, so the peak is SMs x 128 lanes x 2 x clock."""
+    fp32 FMA on the CUDA cores, so the peak is SMs x 128 lanes x 2 x clock.
+
+    With cpu_rows > 0 the fp64 oracle is timed beside it on the first cpu_rows
+    rows of the same problem (an exact sample: rows i < k depend only on the
+    leading k x k block of UL) and scaled by the ratio of multiply-adds."""
     import torch
 
     g = torch.Generator(device=dev).manual_seed(2)
@@ -450,14 +455,47 @@ def measure_gptq2d(gq, dev, clocks, m=4096, n=4096, tokens=8192, reps=5):
     mhz = float((clocks or {}).get("sm_max_mhz") or 1965.0)
     peak = sms * 128 * 2 * mhz * 1e6 / 1e12
     achieved = flops / (ms * 1e-3) / 1e12
-    return {"workload": f"W {m}x{n} fp32 N(0, 0.02); HL, HR Grams of {tokens} N(0,1) tokens, damp 0.01; "
-                        "scale 0.005, codes in [-8, 7]",
+    res = {"workload": f"W {m}x{n} fp32 N(0, 0.02); HL, HR Grams of {tokens} N(0,1) tokens, damp 0.01; "
+                       "scale 0.005, codes in [-8, 7]",
             "kernels": "round2d_tile_kernel + push2d_kernel per tile wavefront",
             "ms_per_call": ms, "launches_per_call": (gq.gptq_kernel_launches() - launches0) / reps,
             "weights_per_s": m * n / (ms * 1e-3),
             "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "algorithmic_flops": flops,
                          "peak_source": f"fp32 FMA: {sms} SMs x 128 lanes x 2 flops x {mhz:.0f} MHz"}}
+    if cpu_rows > 0:
+        res["cpu_baseline"] = gptq2d_oracle_sample(W, U[0], U[1], cpu_rows)
+    return res
+
+
+def gptq2d_oracle_sample(W, UL, UR, k):
+    """fp64 oracle on rows [0, k) of the GPTQ-2D problem, scaled to all rows by
+    the ratio of multiply-adds (sum over entries of (i + 1) + (n - j))."""
+    import numpy as np
+
+    from oracle import gptq2d_oracle as g2
+
+    m, n = W.shape
+    Wh = W[:k].double().cpu().numpy()
+    ULh = UL[:k, :k].double().cpu().numpy()
+    URh = UR.double().cpu().numpy()
+    t0 = time.perf_counter()
+    g2.gptq2d(Wh, ULh, URh, 0.005, -8, 7)
+    dt = time.perf_counter() - t0
+
+    def macs(rows):
+        return n * rows * (rows + 1) / 2 + rows * n * (n + 1) / 2
+
+    scale = macs(m) / macs(k)
+    est = dt * scale
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((i.get("num_threads") or 0) for i in threadpool_info()) or len(os.sched_getaffinity(0))
+    except Exception:
+        cores = len(os.sched_getaffinity(0))
+    return {"value": m * n / est, "unit": "weights/s", "cores": cores, "kind": "oracle",
+            "sample": f"fp64 oracle on the first {k} of {m} rows (all {n} columns) of the same problem, "
+                      f"measured {dt:.2f} s, scaled x{scale:.1f} by multiply-adds"}
 
 
 def run_e2e(args, spec, W, X, dev, world, dist):
