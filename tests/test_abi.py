@@ -105,3 +105,9 @@ def test_gptq2d_arguments_rejected_before_any_launch(lib):
     assert f(fake, 0, 0, 8, fake, fake, 1.0, 0, 0, 0, fake, None, None, 0, None) == 0       # empty: no-op
     assert f(fake, 0, (1 << 22) + 1, 1, fake, fake, 1.0, 0, 0, 0, fake, None, fake, big, None) == 1
 
+
+def test_binding_fails_loudly_without_the_library(tmp_path):
+    from post_weight_quantization_accum_b200 import _lib
+    with pytest.raises(ImportError, match="no fallback"):
+        _lib.load(str(tmp_path / "libgptq_b200.so"))
+
