@@ -12,6 +12,11 @@ Default workload: a Llama-7B attention projection, W 4096x4096 bf16 and X
 N GPUs (torchrun): every rank quantizes its own layer (a different seed); no
 collective on the data path (weak scaling); time = max over ranks.
 
+--workload layerset_block: one step = one block of the 7B-shaped layer set
+(q, k, v, o 4096x4096; gate, up 11008x4096; down 4096x11008; one X of 131,072
+tokens per input group, H and U shared by q/k/v and by gate/up), 4-bit g128;
+the 32-block set takes 32 times a block.
+
 --impl reference times the fp64 CPU oracle (the only reference: the method's
 pages publish no code) on a bounded sample of the same workload.
 """
@@ -371,6 +376,152 @@ def run_ours(args, world, rank, local):
     return result if rank == 0 else None
 
 
+def run_layerset(args, world, rank, local):
+    """One block of the 7B-shaped layer set per step (replicas: rank r
+    quantizes block r).  Per input group: H, U once, then every layer that
+    reads that input (column loop + packing)."""
+    import torch
+
+    import post_weight_quantization_accum_b200 as gq
+    import synth_inputs as si
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    n_tok = args.tokens or 131072
+    inputs, layers = si.layerset_block(rank, n_tok=n_tok)
+    X = {g: si.make_activations(spec, dev) for g, spec in inputs.items()}
+    W = {name: si.make_weights(spec, dev) for name, spec, _ in layers}
+    bits, group, damp, block = 4, 128, 0.01, 128
+    grp = {}
+    for g, spec in inputs.items():
+        n = spec.n
+        grp[g] = {"H": torch.zeros((n, n), dtype=torch.float32, device=dev),
+                  "U": torch.empty((n, n), dtype=torch.float32, device=dev),
+                  "perm": torch.empty(n, dtype=torch.int32, device=dev),
+                  "dead": torch.empty(n, dtype=torch.uint8, device=dev),
+                  "ws_h": gq.workspace(gq.LIB.gptq_hessian_workspace_size(n, n_tok), dev),
+                  "ws_p": gq.workspace(gq.LIB.gptq_prepare_workspace_size(n), dev)}
+    lay = {}
+    for name, spec, g in layers:
+        rows, n = spec.rows, spec.n
+        ng = gq.LIB.gptq_num_groups(n, group)
+        lay[name] = {"g": g,
+                     "out": {"codes": torch.empty((rows, n), dtype=torch.uint8, device=dev),
+                             "scales": torch.empty((rows, ng), dtype=torch.float32, device=dev),
+                             "zeros": torch.empty((rows, ng), dtype=torch.uint8, device=dev),
+                             "g_idx": torch.empty(n, dtype=torch.int32, device=dev)},
+                     "packed": torch.empty((rows, gq.LIB.gptq_packed_words_per_row(n, bits)), dtype=torch.int32,
+                                           device=dev),
+                     "packed_z": torch.empty((rows, gq.LIB.gptq_packed_words_per_row(ng, bits)),
+                                             dtype=torch.int32, device=dev),
+                     "ws_q": gq.workspace(gq.LIB.gptq_quantize_workspace_size(rows, n, block), dev)}
+    stream = torch.cuda.current_stream()
+    stage_names = ("hessian", "prepare_hinv", "quantize_layer", "pack")
+
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
+
+    def step(marks):
+        for g, b in grp.items():
+            b["H"].zero_()
+            e = [ev() for _ in range(3)]
+            e[0].record(stream)
+            gq.gptq_hessian_accum(b["H"], X[g], 2.0 / n_tok, ws=b["ws_h"])
+            e[1].record(stream)
+            gq.gptq_prepare_hinv(b["H"], damp, False, perm=b["perm"], dead=b["dead"], U=b["U"], ws=b["ws_p"])
+            e[2].record(stream)
+            marks.append(("hessian", e[0], e[1]))
+            marks.append(("prepare_hinv", e[1], e[2]))
+            for name, l in lay.items():
+                if l["g"] != g:
+                    continue
+                f = [ev() for _ in range(3)]
+                f[0].record(stream)
+                gq.gptq_quantize_layer(W[name], b["U"], bits, group, block, dead=b["dead"], out=l["out"],
+                                       ws=l["ws_q"])
+                f[1].record(stream)
+                gq.gptq_pack(l["out"]["codes"], bits, packed=l["packed"])
+                gq.gptq_pack(l["out"]["zeros"], bits, packed=l["packed_z"])
+                f[2].record(stream)
+                marks.append(("quantize_layer", f[0], f[1]))
+                marks.append(("pack", f[1], f[2]))
+
+    for _ in range(args.warmup):
+        step([])
+    torch.cuda.synchronize()
+    st = gq.gptq_get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {st}")
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    marks = []
+    t_start, t_end = ev(), ev()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = gq.gptq_kernel_launches()
+    t_start.record(stream)
+    for _ in range(args.steps):
+        step(marks)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    launches = gq.gptq_kernel_launches() - launches0
+    if sampler:
+        time.sleep(0.2)
+        sampler.stop()
+    ms_per_step = max_over_ranks(t_start.elapsed_time(t_end), dist, dev) / args.steps
+    status = gq.gptq_get_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status after the timed region: {status}")
+    stage_ms = {k: sum(a.elapsed_time(b) for s_, a, b in marks if s_ == k) / args.steps for k in stage_names}
+    weights = sum(spec.rows * spec.n for _, spec, _ in layers)
+    value = world * weights / (ms_per_step / 1e3)
+    pk, pk_src = peaks()
+    flops_syrk = sum(float(spec.n) * (spec.n + 1) * n_tok for spec in inputs.values())
+    achieved = flops_syrk / (stage_ms["hessian"] / 1e3) / 1e12
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"layerset_block: one 7B-shaped block (q, k, v, o 4096x4096; gate, up 11008x4096; "
+                               f"down 4096x11008; {weights} weights), X {n_tok} tokens per input group (1% outlier "
+                               f"channels x20), H and U shared by q/k/v and gate/up, 4-bit g128, damp 0.01; "
+                               f"the 32-block set = 32 steps",
+                   "global_batch": n_tok * world, "seq_len": 2048, "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2 (6.1 GB of X per block)",
+                   "timing": "CUDA events on the launching stream; max over ranks"},
+        "roofline": {"bound": "tensor", "kernel": "syrk_tc_kernel (+ its finalize kernel), 4 launches per block",
+                     "achieved": achieved, "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                     "frac": achieved / pk["bf16_tflops_sustained"], "traffic": None,
+                     "peak_source": f"{pk_src} bf16 sustained", "algorithmic_flops": flops_syrk},
+        "stages_ms": stage_ms,
+        "set_seconds_estimate": 32 * ms_per_step / 1e3,
+        "gpu_launches": launches,
+    }
+    if sampler:
+        result["clocks"] = sampler.summary()
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result if rank == 0 else None
+
+
 def measure_matvec(gq, packed, out, spec, dev, pk, copies=16, reps=64):
     """Inference with the layer's packed weights (batch 1, bf16 x), outside the
     timed step: per-launch time over `reps` launches that cycle through
@@ -542,12 +693,72 @@ def run_e2e(args, spec, W, X, dev, world, dist):
 # reference arm: the CPU oracle
 # ---------------------------------------------------------------------------
 
+def reference_layerset_sample():
+    """fp64 oracle estimate for one block of the layer set, from a bounded
+    sample: H on 2048 tokens of a 4096-wide input, the full 4096 x 4096
+    factor, 16 rows of a 4096-column layer through the column loop; each
+    stage scaled to every group and layer by its cost model (H ~ n^2 N,
+    factor ~ n^3, column loop ~ rows n^2)."""
+    import synth_inputs as si
+    from oracle import gptq_oracle as go
+
+    inputs, layers = si.layerset_block(0, n_tok=131072)
+    xs = si.scaled(inputs["qkv"], n_tok=2048)
+    X = si.make_activations(xs, "cpu").double().numpy()
+    ws = [spec for name, spec, _ in layers if name == "q"][0]
+    W = si.make_weights(ws, "cpu")[:16].double().numpy()
+    t0 = time.perf_counter()
+    H = go.hessian(X)
+    t1 = time.perf_counter()
+    prep = go.prepare(H, W, 0.01, False)
+    U = go.inverse_factor(prep["H"])
+    t2 = time.perf_counter()
+    res = go.gptq_quantize(prep["W"], U, 4, 128, 128)
+    go.pack_codes(res["codes"], 4)
+    t3 = time.perf_counter()
+    est = 0.0
+    for spec in inputs.values():
+        r = spec.n / 4096.0
+        est += (t1 - t0) * r * r * (spec.n_tok / 2048.0) + (t2 - t1) * r ** 3
+    for _, spec, _ in layers:
+        r = spec.n / 4096.0
+        est += (t3 - t2) * (spec.rows / 16.0) * r * r
+    weights = sum(spec.rows * spec.n for _, spec, _ in layers)
+    sample = (f"fp64 oracle: H on 2048 of 131072 tokens, the full 4096x4096 factor, 16 rows of q through the loop "
+              f"(measured {t3 - t0:.2f} s), scaled to the block's 4 inputs and 7 layers (H ~ n^2 N, factor ~ n^3, "
+              f"loop ~ rows n^2)")
+    return weights / est, est, sample
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return None
     import torch
 
     import synth_inputs as si
+
+    if args.workload == "layerset_block":
+        vals, ests = [], []
+        for _ in range(args.warmup + args.steps):
+            v, est, sample = reference_layerset_sample()
+            vals.append(v)
+            ests.append(est)
+        vals, ests = vals[args.warmup:], ests[args.warmup:]
+        value = statistics.mean(vals)
+        try:
+            from threadpoolctl import threadpool_info
+            cores = max((i.get("num_threads") or 0) for i in threadpool_info()) or len(os.sched_getaffinity(0))
+        except Exception:
+            cores = len(os.sched_getaffinity(0))
+        cpu = {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+        return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.mean(ests) * 1e3,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic",
+                "config": {"workload": "layerset_block (oracle on a bounded sample, scaled to the block)",
+                           "global_batch": 131072, "seq_len": 2048, "parallelism": "cpu"},
+                "cpu_baseline": cpu,
+                "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
     spec = si.SPECS[args.workload]
     # a bounded sample per step: 2048 tokens for H, 16 rows through the loop
@@ -579,6 +790,8 @@ def main():
     world, rank, local = dist_env()
     if args.impl == "reference":
         res = run_reference(args, world, rank)
+    elif args.workload == "layerset_block":
+        res = run_layerset(args, world, rank, local)
     else:
         res = run_ours(args, world, rank, local)
     if res is not None:

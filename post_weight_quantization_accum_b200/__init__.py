@@ -27,6 +27,7 @@ __all__ = [
     "gptq_kernel_launches",
     "workspace",
     "quantize_layer",
+    "quantize_layer_group",
 ]
 
 
@@ -269,3 +270,42 @@ def quantize_layer(W, X, bits=4, group=128, damp=0.01, block=128, act_order=Fals
     out["packed_zeros"] = gptq_pack(out["zeros"], bits, stream=stream)
     out.update(H=H, U=U, perm=perm, dead=dead)
     return out
+
+
+def quantize_layer_group(Ws, X, bits=4, group=128, damp=0.01, block=128, act_order=False, stream=None,
+                         device=None, chunk_tokens=16384):
+    """Several layers that read the same input (e.g. the q, k and v projections):
+    H, the damping, act-order and U depend only on X, so they are computed once
+    and every layer's column loop and packing reuse them.
+
+    Ws: dict name -> W [rows_i, n]; X: [n_tok, n] bf16 (device or host).
+    Returns dict(H, U, perm, dead, layers={name: outputs as in quantize_layer}).
+    """
+    first = next(iter(Ws.values()))
+    n = first.shape[1]
+    if any(W.shape[1] != n for W in Ws.values()):
+        raise ValueError("every layer of a group must have X's width as its column count")
+    dev = torch.device(device) if device is not None else (first.device if first.is_cuda else
+                                                             torch.device("cuda", torch.cuda.current_device()))
+    H = torch.zeros((n, n), dtype=torch.float32, device=dev)
+    hdiag = torch.zeros(n, dtype=torch.float64, device=dev) if act_order else None
+    if not X.is_cuda:
+        _hessian_from_host(H, X, hdiag, stream, chunk_tokens)
+    else:
+        if X.stride(1) != 1 or X.stride(0) % 8 != 0 or X.data_ptr() % 16 != 0:
+            Xp = torch.zeros((X.shape[0], (n + 7) // 8 * 8), dtype=torch.bfloat16, device=dev)
+            Xp[:, :n] = X
+            X = Xp[:, :n]
+        gptq_hessian_accum(H, X, 2.0 / X.shape[0], hdiag=hdiag, stream=stream)
+    U, perm, dead = gptq_prepare_hinv(H, damp, act_order, hdiag=hdiag, stream=stream)
+    layers = {}
+    for name, W in Ws.items():
+        if not W.is_cuda:
+            W = W.to(dev, non_blocking=True)
+        out = gptq_quantize_layer(W, U, bits, group, block, perm=perm if act_order else None, dead=dead,
+                                  stream=stream)
+        out["packed"] = gptq_pack(out["codes"], bits, stream=stream)
+        out["packed_zeros"] = gptq_pack(out["zeros"], bits, stream=stream)
+        layers[name] = out
+    return {"H": H, "U": U, "perm": perm, "dead": dead, "layers": layers}
+

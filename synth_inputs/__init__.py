@@ -114,3 +114,24 @@ def make_activations(spec, device="cpu", chunk=16384):
 
 def make_layer(spec, device="cpu"):
     return make_weights(spec, device), make_activations(spec, device)
+
+
+def layerset_block(block, n_tok=131072, bits=4, group=128):
+    """One block of the 7B-shaped layer set: the four calibration inputs (one
+    per input group, 1% outlier channels x20) and the seven weight matrices.
+
+    Returns (inputs, layers): inputs maps an input group to the LayerSpec of
+    its activations (rows unused); layers lists (name, LayerSpec of the
+    weights, input group).  Seeds: input group g of block b uses 40000 + 4b + g
+    (its activations draw from that + 1000), layer i uses 50000 + 8b + i.
+    """
+    groups = ["qkv", "o", "gateup", "down"]
+    widths = {"qkv": 4096, "o": 4096, "gateup": 4096, "down": 11008}
+    inputs = {g: LayerSpec(f"layerset.b{block}.{g}", 0, widths[g], n_tok, bits=bits, group=group,
+                           seed=40000 + 4 * block + gi)
+              for gi, g in enumerate(groups)}
+    layers = [(name, LayerSpec(f"layerset.b{block}.{name}", rows, n, n_tok, bits=bits, group=group,
+                               seed=50000 + 8 * block + i), g)
+              for i, (name, rows, n, g) in enumerate(LAYERSET_BLOCK)]
+    return inputs, layers
+
