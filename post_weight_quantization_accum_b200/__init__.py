@@ -189,6 +189,12 @@ def gptq2d_round(W, UL, UR, scale=1.0, qmin=None, qmax=None, want_E=True, codes=
     dev = W.device
     if (qmin is None) != (qmax is None):
         raise ValueError("give both qmin and qmax, or neither")
+    if tuple(UL.shape) != (m, m) or tuple(UR.shape) != (n, n):
+        raise ValueError(f"factors {tuple(UL.shape)} and {tuple(UR.shape)} do not match W {tuple(W.shape)}")
+    if UL.dtype != torch.float32 or UR.dtype != torch.float32:
+        raise TypeError("UL and UR must be fp32")
+    if not (W.is_contiguous() and UL.is_contiguous() and UR.is_contiguous()):
+        raise ValueError("W, UL and UR must be contiguous row-major matrices")
     clamp = 0 if qmin is None else 1
     codes = codes if codes is not None else torch.empty((m, n), dtype=torch.int32, device=dev)
     if want_E and E is None:

@@ -111,3 +111,17 @@ def test_binding_fails_loudly_without_the_library(tmp_path):
     with pytest.raises(ImportError, match="no fallback"):
         _lib.load(str(tmp_path / "libgptq_b200.so"))
 
+
+
+def test_gptq2d_binding_checks_shapes_before_the_library():
+    import torch
+    import post_weight_quantization_accum_b200 as gq
+    W = torch.zeros((3, 5))
+    with pytest.raises(ValueError):
+        gq.gptq2d_round(W, torch.eye(3), torch.eye(4))
+    with pytest.raises(TypeError):
+        gq.gptq2d_round(W, torch.eye(3, dtype=torch.float64), torch.eye(5))
+    with pytest.raises(ValueError):
+        gq.gptq2d_round(W, torch.eye(3), torch.eye(6)[:5, :5])   # a non-contiguous view
+    with pytest.raises(ValueError):
+        gq.gptq2d_round(W, torch.eye(3), torch.eye(5), qmin=-1)
