@@ -28,6 +28,7 @@
 // with J L J upper triangular, so U = (J L J)^-1 = J L^-1 J is upper with
 // U^T U = H'^-1: it is the upper Cholesky factor of the inverse.
 #include <algorithm>
+#include <atomic>
 
 #include "common.cuh"
 
@@ -656,7 +657,7 @@ PrepLayout prep_layout(int n) {
 }
 
 int chol_grid(const DeviceInfo* info) {
-  static int blocks_per_sm[64] = {};
+  static std::atomic<int> blocks_per_sm[64] = {};  // per device, shared by host threads
   if (blocks_per_sm[info->device] == 0) {
     int b = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, chol_inv_kernel, kCholThreads, kCholSmem) != cudaSuccess ||
@@ -693,7 +694,7 @@ gptq_status prepare_hinv(const float* H, const double* hdiag, int n, float damp,
   int32_t* perm = perm_out != nullptr ? perm_out : reinterpret_cast<int32_t*>(w + l.perm);
   int* fstatus = info->status + 1;
 
-  static bool attr_set[64] = {};
+  static std::atomic<bool> attr_set[64] = {};  // per device, shared by host threads
   if (!attr_set[info->device]) {
     if (cudaFuncSetAttribute(chol_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kCholSmem)) != cudaSuccess)

@@ -21,6 +21,7 @@
 // x computed once per CTA.  Otherwise (act-order g_idx, or groups that split
 // runs) every code looks up its own scale and zero point.
 #include <algorithm>
+#include <atomic>
 
 #include "common.cuh"
 
@@ -202,7 +203,7 @@ gptq_status launch_matvec(const uint32_t* packed, const float* scales, const uin
   const DeviceInfo* info = device_info();
   if (info == nullptr) return GPTQ_ERR_CUDA;
   const size_t smem = smem_bytes(B);
-  static bool attr_set[64] = {};
+  static std::atomic<bool> attr_set[64] = {};  // per device, shared by host threads
   if (!attr_set[info->device]) {
     if (cudaFuncSetAttribute(dequant_matvec_kernel<BITS, B, kFast, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)

@@ -27,6 +27,7 @@
 //                       tf32 split; the block kernel writes E as its tf32
 //                       hi / lo halves.
 #include <algorithm>
+#include <atomic>
 #include <cstring>
 
 #include "common.cuh"
@@ -414,7 +415,7 @@ gptq_status quantize_layer(const void* W, gptq_dtype wdt, int64_t rows, int n, c
   const int64_t want = ceil_div(warps_needed, static_cast<int64_t>(2 * info->sm_count));
   const int warps_per_cta = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(kMaxWarpsPerCta, want)));
   const unsigned block_ctas = static_cast<unsigned>(ceil_div(warps_needed, static_cast<int64_t>(warps_per_cta)));
-  static bool attr_set[64] = {};
+  static std::atomic<bool> attr_set[64] = {};  // per device, shared by host threads
   if (!attr_set[info->device]) {
     if (cudaFuncSetAttribute(gptq_block_kernel<kBlockLanes>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(block_smem)) != cudaSuccess)

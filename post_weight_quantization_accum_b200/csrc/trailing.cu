@@ -27,6 +27,7 @@
 // Every barrier wait is bounded; on a timeout the CTA drains its own copies
 // and MMAs and returns with GPTQ_ERR_TIMEOUT recorded.
 #include <algorithm>
+#include <atomic>
 
 #include "common.cuh"
 
@@ -334,7 +335,7 @@ __global__ void split_cols_tf32_kernel(const float* __restrict__ src, int64_t ld
 }
 
 bool set_smem_attr(const DeviceInfo* info) {
-  static bool attr_set[64] = {};
+  static std::atomic<bool> attr_set[64] = {};  // per device, shared by host threads
   if (!attr_set[info->device]) {
     if (cudaFuncSetAttribute(trailing_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemBytes)) != cudaSuccess)
