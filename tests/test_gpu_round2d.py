@@ -122,6 +122,18 @@ def test_round2d_deterministic():
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
 
 
+def test_round2d_without_error_output():
+    # E = NULL: the errors live in the workspace; the codes are the same
+    W, UL, UR = _inputs(60, 130, 190)
+    dev = "cuda"
+    args = (torch.tensor(W, device=dev), torch.tensor(UL, device=dev), torch.tensor(UR, device=dev), 0.25)
+    a = gq.gptq2d_round(*args)
+    b = gq.gptq2d_round(*args, want_E=False)
+    torch.cuda.synchronize()
+    assert b["E"] is None
+    assert torch.equal(a["codes"], b["codes"])
+
+
 def test_round2d_full_size_sampled():
     """W 4096 x 4096 (N(0, 0.02)), a 4-bit signed grid (scale 0.005, codes in
     [-8, 7]); HL and HR are Grams of 8192 N(0, 1) tokens built and factored by
