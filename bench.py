@@ -83,6 +83,27 @@ def job_rate(world, rows, n, ms):
     return world * rows * n / (ms / 1e3)
 
 
+def stage_rooflines(stage_ms, rows, n, bits, ng, sms, mhz, hbm_gbs):
+    """Roofline fractions of the non-SYRK stages from their CUDA-event times.
+
+    factorization: 2 n^3 / 3 flops of fp32 FMA work on the CUDA cores against
+    SMs x 128 lanes x 2 flops x clock; packing: the codes and zero points read
+    (1 byte each) and their packed words written, against the HBM copy rate.
+    """
+    t_factor = stage_ms["prepare_hinv"] / 1e3
+    t_pack = stage_ms["pack"] / 1e3
+    alu_peak = sms * 128 * 2 * mhz * 1e6 / 1e12
+    factor_tflops = 2.0 * n ** 3 / 3.0 / t_factor / 1e12
+    words = lambda k: bits * ((k + 31) // 32)
+    pack_bytes = rows * n + rows * ng + 4 * rows * (words(n) + words(ng))
+    pack_gbs = pack_bytes / t_pack / 1e9
+    return {"factorization": {"bound": "alu", "achieved": factor_tflops, "peak": alu_peak, "unit": "TFLOP/s",
+                              "frac": factor_tflops / alu_peak,
+                              "peak_source": f"fp32 FMA: {sms} SMs x 128 lanes x 2 flops x {mhz:.0f} MHz"},
+            "pack": {"bound": "hbm", "achieved": pack_gbs, "peak": hbm_gbs, "unit": "GB/s",
+                     "frac": pack_gbs / hbm_gbs, "algorithmic_bytes": pack_bytes}}
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -357,6 +378,10 @@ def run_ours(args, world, rank, local):
     }
     if sampler:
         result["clocks"] = sampler.summary()
+    result["stage_rooflines"] = stage_rooflines(
+        dict(zip(("hessian", "prepare_hinv", "quantize_layer", "pack"), stage_ms)), rows, n, spec.bits, ng,
+        torch.cuda.get_device_properties(dev).multi_processor_count,
+        float((result.get("clocks") or {}).get("sm_max_mhz") or 1965.0), pk["hbm_gbs"])
     result["packed_matvec"] = measure_matvec(gq, packed, out, spec, dev, pk)
     if not args.no_gptq2d:
         cpu_rows = 64 if (world == 1 and rank == 0 and not args.no_cpu_baseline) else 0

@@ -26,3 +26,15 @@ def test_reference_arm_prints_one_contract_line():
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     assert d["e2e"]["value"] == d["value"] and d["e2e"]["h2d_bytes_per_step"] == 0
     assert d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_stage_rooflines_arithmetic():
+    sys.path.insert(0, ROOT)
+    import bench
+    r = bench.stage_rooflines({"hessian": 3.0, "prepare_hinv": 2.0, "quantize_layer": 1.0, "pack": 0.01},
+                              rows=4096, n=4096, bits=4, ng=32, sms=148, mhz=2000.0, hbm_gbs=6000.0)
+    assert abs(r["factorization"]["peak"] - 148 * 256 * 2.0e9 / 1e12) < 1e-9
+    assert abs(r["factorization"]["achieved"] - 2 * 4096 ** 3 / 3 / 2e-3 / 1e12) < 1e-6
+    # codes and zeros read (1 byte each), 512 + 4 packed words per row written
+    assert r["pack"]["algorithmic_bytes"] == 4096 * 4096 + 4096 * 32 + 4 * 4096 * (512 + 4)
+    assert abs(r["pack"]["frac"] - r["pack"]["achieved"] / 6000.0) < 1e-12
