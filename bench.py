@@ -365,9 +365,10 @@ def run_ours(args, world, rank, local):
                    "l2": "inputs larger than L2 (X alone is %.2f GB)" % (spec.n_tok * n * 2 / 1e9),
                    "timing": "CUDA events on the launching stream; max over ranks"},
         "roofline": {"bound": "tensor", "kernel": "syrk_tc_kernel (+ its finalize kernel)", "achieved": achieved,
-                     "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                     "frac": achieved / pk["bf16_tflops_sustained"], "traffic": traffic,
-                     "peak_source": f"{pk_src} bf16 sustained (kernel timed inside a long step)",
+                     "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / pk["bf16_tflops"], "traffic": traffic,
+                     "peak_source": f"{pk_src} bf16 burst (the call is timed alone with CUDA events, a few ms)",
+                     "frac_of_sustained": achieved / pk["bf16_tflops_sustained"],
                      "algorithmic_flops": flops_syrk},
         "stages_ms": {"hessian": stage_ms[0], "prepare_hinv": stage_ms[1], "quantize_layer": stage_ms[2],
                       "pack": stage_ms[3]},
@@ -532,9 +533,10 @@ def run_layerset(args, world, rank, local):
                    "l2": "inputs larger than L2 (6.1 GB of X per block)",
                    "timing": "CUDA events on the launching stream; max over ranks"},
         "roofline": {"bound": "tensor", "kernel": "syrk_tc_kernel (+ its finalize kernel), 4 launches per block",
-                     "achieved": achieved, "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                     "frac": achieved / pk["bf16_tflops_sustained"], "traffic": None,
-                     "peak_source": f"{pk_src} bf16 sustained", "algorithmic_flops": flops_syrk},
+                     "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / pk["bf16_tflops"], "traffic": None,
+                     "peak_source": f"{pk_src} bf16 burst (each call timed alone with CUDA events)",
+                     "frac_of_sustained": achieved / pk["bf16_tflops_sustained"], "algorithmic_flops": flops_syrk},
         "stages_ms": stage_ms,
         "set_seconds_estimate": 32 * ms_per_step / 1e3,
         "gpu_launches": launches,

@@ -233,6 +233,9 @@ gptq_status gptq_quantize_layer(const void* W, gptq_dtype wdt, int64_t rows,
  *     (e.g. 1024 x 1024 fits, 1024 x 2048 does not).
  *   - The first call on a device looks up the array's device address (with
  *     that device current); make that first call before any stream capture.
+ *     The address is kept for the life of the process: after cudaDeviceReset
+ *     (or in another context on the same device) it is stale, so do not call
+ *     this entry point again in that process after a reset.
  *   - All calls share the array: calls whose kernels overlap on the GPU race
  *     and give wrong results.  The array keeps the last call's contents; the
  *     column loop writes every scratch byte before reading it.

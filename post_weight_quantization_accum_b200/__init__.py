@@ -21,6 +21,7 @@ __all__ = [
     "gptq_pack",
     "gptq_dequant_matvec",
     "gptq2d_round",
+    "gptq2d_check_args",
     "gptq2d_factor",
     "gptq_get_device_status",
     "gptq_set_wait_limit_ns",
@@ -179,22 +180,32 @@ def gptq2d_factor(H, damp=0.0, ws=None, stream=None):
     return U
 
 
+def gptq2d_check_args(W, UL, UR, qmin=None, qmax=None):
+    """The checks gptq2d_round makes before it touches the device (shapes,
+    dtypes, row-major layout); they need no GPU, so callers can run them on
+    host tensors built the same way."""
+    m, n = W.shape
+    if (qmin is None) != (qmax is None):
+        raise ValueError("give both qmin and qmax, or neither")
+    if tuple(UL.shape) != (m, m) or tuple(UR.shape) != (n, n):
+        raise ValueError(f"factors {tuple(UL.shape)} and {tuple(UR.shape)} do not match W {tuple(W.shape)}")
+    if W.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError(f"unsupported weight dtype {W.dtype}")
+    if UL.dtype != torch.float32 or UR.dtype != torch.float32:
+        raise TypeError("UL and UR must be fp32")
+    if not (W.is_contiguous() and UL.is_contiguous() and UR.is_contiguous()):
+        raise ValueError("W, UL and UR must be contiguous row-major matrices")
+
+
 def gptq2d_round(W, UL, UR, scale=1.0, qmin=None, qmax=None, want_E=True, codes=None, E=None, ws=None,
                  stream=None):
     """Two-sided GPTQ (GPTQ-2D): round W [m, n] (fp32 or bf16) to scale * integers
     under tr(HL D HR D^T), given the upper factors UL (UL^T UL = HL^-1) and UR
     (UR^T UR = HR^-1).  Clamps the integers to [qmin, qmax] when both are given.
     Returns dict(codes=int32 [m, n], E=fp32 [m, n] scaled errors or None)."""
+    gptq2d_check_args(W, UL, UR, qmin, qmax)
     m, n = W.shape
     dev = W.device
-    if (qmin is None) != (qmax is None):
-        raise ValueError("give both qmin and qmax, or neither")
-    if tuple(UL.shape) != (m, m) or tuple(UR.shape) != (n, n):
-        raise ValueError(f"factors {tuple(UL.shape)} and {tuple(UR.shape)} do not match W {tuple(W.shape)}")
-    if UL.dtype != torch.float32 or UR.dtype != torch.float32:
-        raise TypeError("UL and UR must be fp32")
-    if not (W.is_contiguous() and UL.is_contiguous() and UR.is_contiguous()):
-        raise ValueError("W, UL and UR must be contiguous row-major matrices")
     clamp = 0 if qmin is None else 1
     codes = codes if codes is not None else torch.empty((m, n), dtype=torch.int32, device=dev)
     if want_E and E is None:
@@ -240,8 +251,17 @@ def _hessian_from_host(H, X, hdiag, stream, chunk_tokens):
     return H
 
 
+def _raise_on_device_status(stream):
+    # A bounded in-kernel wait that ran out leaves the asynchronous calls'
+    # status at GPTQ_OK but records GPTQ_ERR_TIMEOUT on the device; read (and
+    # clear) it so that such a run cannot hand back wrong codes silently.
+    code = gptq_get_device_status(stream)
+    if code != 0:
+        raise GptqError("device status", code)
+
+
 def quantize_layer(W, X, bits=4, group=128, damp=0.01, block=128, act_order=False, want_deq=False,
-                   want_loss=False, stream=None, device=None, chunk_tokens=16384):
+                   want_loss=False, stream=None, device=None, chunk_tokens=16384, check=True):
     """One linear layer end to end: H from X, U, the column loop, packing.
 
     W: [rows, n] fp32/bf16 weights; X: [n_tok, n] bf16 calibration inputs.
@@ -250,7 +270,9 @@ def quantize_layer(W, X, bits=4, group=128, damp=0.01, block=128, act_order=Fals
     copy of the next.  Everything is computed on `device` (default: W's device
     if W is on a GPU, else the current one).  Returns a dict of device tensors
     with H, U, perm, codes, scales, zeros, g_idx, packed, packed_zeros (and deq
-    / row_loss when asked for).
+    / row_loss when asked for).  With ``check`` (the default) the call ends by
+    reading the library's device status word, which synchronizes the stream,
+    and raises GptqError if a bounded in-kernel wait ran out.
     """
     n = W.shape[1]
     dev = torch.device(device) if device is not None else (W.device if W.is_cuda else
@@ -275,17 +297,20 @@ def quantize_layer(W, X, bits=4, group=128, damp=0.01, block=128, act_order=Fals
     out["packed"] = gptq_pack(out["codes"], bits, stream=stream)
     out["packed_zeros"] = gptq_pack(out["zeros"], bits, stream=stream)
     out.update(H=H, U=U, perm=perm, dead=dead)
+    if check:
+        _raise_on_device_status(stream)
     return out
 
 
 def quantize_layer_group(Ws, X, bits=4, group=128, damp=0.01, block=128, act_order=False, stream=None,
-                         device=None, chunk_tokens=16384):
+                         device=None, chunk_tokens=16384, check=True):
     """Several layers that read the same input (e.g. the q, k and v projections):
     H, the damping, act-order and U depend only on X, so they are computed once
     and every layer's column loop and packing reuse them.
 
     Ws: dict name -> W [rows_i, n]; X: [n_tok, n] bf16 (device or host).
-    Returns dict(H, U, perm, dead, layers={name: outputs as in quantize_layer}).
+    Returns dict(H, U, perm, dead, layers={name: outputs as in quantize_layer});
+    ``check`` as in quantize_layer.
     """
     first = next(iter(Ws.values()))
     n = first.shape[1]
@@ -313,5 +338,7 @@ def quantize_layer_group(Ws, X, bits=4, group=128, damp=0.01, block=128, act_ord
         out["packed"] = gptq_pack(out["codes"], bits, stream=stream)
         out["packed_zeros"] = gptq_pack(out["zeros"], bits, stream=stream)
         layers[name] = out
+    if check:
+        _raise_on_device_status(stream)
     return {"H": H, "U": U, "perm": perm, "dead": dead, "layers": layers}
 

@@ -44,7 +44,7 @@ constexpr uint64_t kDefaultWaitNs = 2000000000ull;
 std::mutex g_mutex;
 DeviceInfo g_info[kMaxDevices];
 bool g_have[kMaxDevices] = {};
-uint64_t g_wait_ns = kDefaultWaitNs;
+std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};  // read by every launch, set from any thread
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -100,7 +100,7 @@ bool make_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void*
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-uint64_t wait_limit_ns() { return g_wait_ns; }
+uint64_t wait_limit_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
 
 static std::atomic<uint64_t> g_launches{0};
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
@@ -135,7 +135,9 @@ int32_t gptq_version(void) { return 100; }
 
 uint64_t gptq_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
-void gptq_set_wait_limit_ns(uint64_t ns) { g_wait_ns = ns == UINT64_MAX ? 2000000000ull : ns; }
+void gptq_set_wait_limit_ns(uint64_t ns) {
+  g_wait_ns.store(ns == UINT64_MAX ? kDefaultWaitNs : ns, std::memory_order_relaxed);
+}
 
 gptq_status gptq_get_device_status(void* stream) {
   const DeviceInfo* info = device_info();

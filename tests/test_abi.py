@@ -125,3 +125,16 @@ def test_gptq2d_binding_checks_shapes_before_the_library():
         gq.gptq2d_round(W, torch.eye(3), torch.eye(6)[:5, :5])   # a non-contiguous view
     with pytest.raises(ValueError):
         gq.gptq2d_round(W, torch.eye(3), torch.eye(5), qmin=-1)
+
+
+def test_smoke_gptq2d_inputs_pass_the_binding_checks():
+    """smoke() builds its GPTQ-2D inputs with the oracle's factor and
+    torch.tensor; the same construction on the host must satisfy every check
+    gptq2d_round makes before it touches the device (a non-contiguous factor
+    once failed smoke on the GPU)."""
+    import __graft_entry__ as ge
+    import post_weight_quantization_accum_b200 as gq
+    W2, UL, UR = ge.gptq2d_smoke_inputs()
+    W, ULt, URt = ge.gptq2d_smoke_tensors(W2, UL, UR, "cpu")
+    assert ULt.is_contiguous() and URt.is_contiguous()
+    gq.gptq2d_check_args(W, ULt, URt)

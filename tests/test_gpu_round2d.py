@@ -40,8 +40,10 @@ def _spd(rng, k, cond):
 
 def _inputs(seed, m, n, cond=30.0):
     rng = np.random.default_rng(seed)
-    UL = go.inverse_factor(_spd(rng, m, cond)).astype(np.float32)
-    UR = go.inverse_factor(_spd(rng, n, cond)).astype(np.float32)
+    # the binding takes row-major (C-contiguous) factors; the oracle's factor
+    # is a transposed view, so copy it into row-major order
+    UL = np.ascontiguousarray(go.inverse_factor(_spd(rng, m, cond)), dtype=np.float32)
+    UR = np.ascontiguousarray(go.inverse_factor(_spd(rng, n, cond)), dtype=np.float32)
     W = rng.standard_normal((m, n)).astype(np.float32)
     return W, UL, UR
 

@@ -10,7 +10,7 @@ from oracle import gptq_oracle as go
 
 
 def test_group_computes_h_and_u_once_and_quantizes_every_layer(monkeypatch):
-    calls = {"h": 0, "p": 0, "q": [], "pack": 0}
+    calls = {"h": 0, "p": 0, "q": [], "pack": 0, "status": 0}
     rng = np.random.default_rng(3)
     n, n_tok = 48, 300
     X = torch.from_numpy(rng.standard_normal((n_tok, n)).astype(np.float32)).to(torch.bfloat16)
@@ -43,8 +43,15 @@ def test_group_computes_h_and_u_once_and_quantizes_every_layer(monkeypatch):
     monkeypatch.setattr(gq, "gptq_prepare_hinv", prepare)
     monkeypatch.setattr(gq, "gptq_quantize_layer", quantize)
     monkeypatch.setattr(gq, "gptq_pack", pack)
+
+    def status(stream=None):
+        calls["status"] += 1
+        return 0
+
+    monkeypatch.setattr(gq, "gptq_get_device_status", status)
     out = gq.quantize_layer_group(Ws, X, bits=3, group=16, damp=0.01, block=16, device="cpu")
     assert calls["h"] == 1 and calls["p"] == 1 and calls["pack"] == 2 * len(Ws)
+    assert calls["status"] == 1  # the device status word is read once, at the end
     assert len(calls["q"]) == len(Ws) and all(U is out["U"] for U in calls["q"])
     for name, W in Ws.items():
         ref = go.gptq_layer(W.double().numpy(), X=X.double().numpy(), bits=3, group=16, damp=0.01, block=16)
