@@ -6,27 +6,16 @@
 // inverse of H):
 //
 //   A = J P^T (H + lambda I) P J          (J = order reversal, P = act-order)
-//   A = L L^T,  X = L^-1                  blocked, see below
-//   U = J X J                             (a reversal of X's storage)
-//
-// Below n = 8192 one persistent cooperative kernel factors A and builds X in
-// 64-wide panels on the CUDA cores.  From there on the same kernel handles
-// each 1024 x 1024 diagonal block, and everything between blocks is a
-// tensor-core GEMM with the fp32-accurate 3-term tf32 split (trailing.cu):
-// for block K (rows and columns [k0, k1)), R the rows of X still being
-// formed,
-//   X_K,<K  = X_KK R_K,<K                 finalize block row K of X
-//   L_>K,K  = A_>K,K X_KK^T               panel (trsm as a product)
-//   A_>K,>K -= L_>K,K L_>K,K^T            trailing update (full square, which
-//                                         also keeps the diagonal tiles' upper
-//                                         halves the factorization reads)
-//   R_>K,<=K -= L_>K,K X_K,<=K            inverse update
-// so the O(n^3) work runs at tensor-core rate and only the 1024-wide diagonal
-// blocks go through the latency-bound panel sweep.
+//   A = L L^T,  X = L^-1                  128-wide panels, see below
+//   U = J X J                             (an anti-transpose of Y = X^T)
 //
 // With H' = P^T (H + lambda I) P, J H' J = L L^T gives H' = (J L J)(J L J)^T
 // with J L J upper triangular, so U = (J L J)^-1 = J L^-1 J is upper with
 // U^T U = H'^-1: it is the upper Cholesky factor of the inverse.
+//
+// A is held at a padded order np (a multiple of 128) with the identity in the
+// padding, so every tile is a whole 128 x 128 tile; the padding's factor and
+// inverse are the identity and never touch the leading n x n block.
 #include <algorithm>
 #include <atomic>
 
@@ -34,7 +23,6 @@
 
 namespace gptq {
 namespace {
-
 
 // --------------------------------------------------------------------------
 // dead columns, damping and the act-order key
@@ -92,39 +80,52 @@ __global__ void identity_perm_kernel(int32_t* perm, int n) {
   if (i < n) perm[i] = i;
 }
 
-constexpr int kT = 64;  // tile width = panel width of the factorization below
-
-// Lower triangle of A = J P^T (H + lambda I) P J; dead diagonals become 1 + lambda.
-// Inside the kT x kT diagonal blocks the upper half is written too, as the
-// mirror of the lower one (the diagonal factorization reads whole blocks).
+// A's lower triangle at the padded order np: the damped, permuted and
+// reversed Hessian where a, b < n, the identity in the padding.  Dead
+// diagonals become 1 + lambda.  (The upper triangle is never read.)
 __global__ void gather_reversed_kernel(const float* __restrict__ H, const int32_t* __restrict__ perm,
                                        const uint8_t* __restrict__ dead, const double* __restrict__ lambda, int n,
-                                       float* __restrict__ A) {
-  const int b = blockIdx.x * blockDim.x + threadIdx.x;
-  const int a = blockIdx.y;
-  if (a >= n || b >= n) return;
-  if (b > a && b / kT != a / kT) return;
-  const int lo = b > a ? a : b, hi = b > a ? b : a;  // the lower-triangle entry (hi, lo) holds the value
-  const int ph = perm[n - 1 - hi], pl = perm[n - 1 - lo];
-  float v;
-  if (a == b) {
-    const double base = dead[ph] ? 1.0 : static_cast<double>(H[static_cast<size_t>(ph) * n + ph]);
-    v = static_cast<float>(base + *lambda);
-  } else {
-    v = H[static_cast<size_t>(ph) * n + pl];
+                                       int64_t np, float* __restrict__ A) {
+  for (int64_t a = blockIdx.y; a < np; a += gridDim.y) {
+    const int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (b > a) continue;
+    float v;
+    if (a < n && b < n) {
+      const int ph = perm[n - 1 - a], pl = perm[n - 1 - b];
+      if (a == b) {
+        const double base = dead[ph] ? 1.0 : static_cast<double>(H[static_cast<size_t>(ph) * n + ph]);
+        v = static_cast<float>(base + *lambda);
+      } else {
+        v = H[static_cast<size_t>(ph) * n + pl];
+      }
+    } else {
+      v = a == b ? 1.0f : 0.0f;
+    }
+    A[a * np + b] = v;
   }
-  A[static_cast<size_t>(a) * n + b] = v;
 }
 
-// U = J X J for X stored row-major in U's own memory: U[a][b] = X[n-1-a][n-1-b]
-// is the reversal of the flat array (element e <-> n*n - 1 - e).
-__global__ void reverse_kernel(float* __restrict__ U, int64_t count) {
-  const int64_t half = count / 2;
-  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < half;
-       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const float a = U[e], b = U[count - 1 - e];
-    U[e] = b;
-    U[count - 1 - e] = a;
+// U[a][b] = Y[n-1-b][n-1-a] (a, b < n): the anti-transpose of Y = X^T, i.e.
+// U = J X J.  32 x 32 tiles through shared memory; tiles strictly below the
+// diagonal are zeros and read nothing.
+__global__ void anti_transpose_kernel(const float* __restrict__ Y, int64_t ldy, int n, float* __restrict__ U) {
+  __shared__ float t[32][33];
+  const int a0 = blockIdx.y * 32, b0 = blockIdx.x * 32;
+  if (b0 + 31 < a0) {
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+      const int a = a0 + i, b = b0 + threadIdx.x;
+      if (a < n && b < n) U[static_cast<int64_t>(a) * n + b] = 0.0f;
+    }
+    return;
+  }
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int b = b0 + i, a = a0 + threadIdx.x;
+    t[i][threadIdx.x] = (a < n && b < n) ? Y[static_cast<int64_t>(n - 1 - b) * ldy + (n - 1 - a)] : 0.0f;
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int a = a0 + i, b = b0 + threadIdx.x;
+    if (a < n && b < n) U[static_cast<int64_t>(a) * n + b] = t[threadIdx.x][i];
   }
 }
 
@@ -132,159 +133,62 @@ __global__ void reverse_kernel(float* __restrict__ U, int64_t count) {
 // Cholesky and inverse in one persistent cooperative kernel
 // --------------------------------------------------------------------------
 //
-// A = L L^T is factored in 64-wide panels; X = L^-1 is built alongside it by
-// a right-looking forward substitution, R_i = I_i - sum_{m<k} L_im X_m:
+// A = L L^T is factored in 128-wide panels k = 0 .. nb-1 while X = L^-1 is
+// built by a right-looking forward substitution (R = I; block row k of X is
+// Linv_kk R_k,<=k, then R_i,<=k -= L_ik X_k,<=k for i > k).  The kernel keeps
+// Y = X^T instead of X (and Ry = R^T in Y's places), which makes every tile
+// product C = P Q^T with both P and Q read along their rows:
 //
-//   phase T(k)  trsm      L_ik = A_ik Linv_kk^T              for i > k
-//               finalize  X_kj = Linv_kk R_kj                for j < k
-//   phase U(k)  update    A_ij -= L_ik L_jk^T                for k < j <= i
-//               inverse   R_ij -= L_ik X_kj                  for i > k, j <= k
-//               factor    L_{k+1,k+1}, Linv_{k+1,k+1}         (by the CTA that
-//                         updated that tile first in the phase)
+//   phase T(k)  trsm      L_ik   = A_ik Linv_kk^T           i > k
+//               finalize  Y_jk   = Ry_jk Linv_kk^T          j < k
+//   phase U(k)  update    A_ij  -= L_ik L_jk^T              k < j <= i
+//               inverse   Ry_ji -= Y_jk L_ik^T              j <= k < i
+//               factor    Linv_{k+1,k+1} and Y_{k+1,k+1}    (CTA 0, right
+//                         after its own update of that tile)
 //
-// Every step is a 64 x 64 x 64 tile product, and the Cholesky half of a phase
-// shrinks as the inverse half grows, so each phase has about the same number
-// of tiles.  Two grid barriers per panel (time-bounded).  The kernel works on
-// one diagonal block of order <= 1024 at any row pitch; R's tiles live in X's
-// places before they are finalized.
+// Every operation is one 128 x 128 x 128 product on the tensor cores
+// (tcgen05.mma kind::tf32, fp32 accumulation in tensor memory), fp32-accurate
+// through the 3-term split P_hi Q_hi + P_hi Q_lo + P_lo Q_hi (x_hi = x with
+// its 13 low mantissa bits cleared, x_lo = x - x_hi; the dropped P_lo Q_lo is
+// below 2^-20 of the product).  Operands are staged through registers (the
+// loads of the next 32-column chunk in flight while the current one is split
+// and stored) into a two-stage shared-memory ring in the 128-byte-swizzled
+// K-major layout; one thread issues the MMAs; the accumulator is
+// double-buffered, so one operation's epilogue (tensor memory -> registers ->
+// a store, or an L2 vector reduction for the subtracting operations) overlaps
+// the next one's products.  Each tile receives at most one result per phase.
+// Two time-bounded grid barriers per panel; every wait is bounded, and a CTA
+// that gives up lets its own tensor-core work finish and releases its tensor
+// memory before returning.
 
-constexpr int kPad = 68;           // shared-memory row stride (16-byte aligned rows)
+constexpr int kT = 128;                      // panel width and tile order
+constexpr int kCk = 32;                      // fp32 columns of K per staged chunk (one 128-byte row)
+constexpr int kChunks = kT / kCk;
 constexpr int kCholThreads = 256;
-constexpr int kMaxCholCtas = 4096;  // bound on the cooperative grid (SM ids recorded per CTA)
-constexpr size_t kCholSmem = 3 * kT * kPad * sizeof(float);
+constexpr int kBufBytes = kT * kCk * 4;      // one split half of one operand chunk (16 KB)
+constexpr int kStageBytes = 4 * kBufBytes;   // P hi, P lo, Q hi, Q lo
+constexpr int kStages = 2;
+constexpr int kSP = 132;                     // row pitch (floats) of the diagonal factor's matrices
+constexpr int kSub = 16;                     // sub-panel width of the diagonal factor
+constexpr size_t kRingBytes = static_cast<size_t>(kStages) * kStageBytes;
+constexpr size_t kFactorBytes = (2 * static_cast<size_t>(kT) * kSP + static_cast<size_t>(kSub) * kT + kT) * 4;
+constexpr size_t kRegionBytes = kFactorBytes > kRingBytes ? kFactorBytes : kRingBytes;
+constexpr size_t kCholSmem = 1024 + kRegionBytes + 128;  // 1024-byte alignment slack, region, barriers
+constexpr uint32_t kCholTmemCols = 2 * kT;               // two 128 x 128 fp32 accumulators
+constexpr int kMaxCholCtas = 1024;
+constexpr uint64_t kDrainNs = 2000000000ull;
 
 struct CholArgs {
-  float* A;          // block [n, n] at row pitch lda, lower: the damped reversed matrix, becomes L
-  float* X;          // block [n, n] at row pitch ldx, zero on entry: X = L^-1 is written here
-  int64_t lda, ldx;
-  int n;             // order of the block
-  int nblk;
-  int* fstatus;      // factorization status word
-  unsigned* bar;     // grid barrier: [0] arrivals, [1] generation (zeroed on entry)
-  int* abort;        // set when a barrier wait runs out (zeroed on entry)
+  float* A;         // [np, np] at pitch ld, lower: the damped reversed matrix; panels become L
+  float* Y;         // [np, np] at pitch ld, zero on entry: becomes Y = (L^-1)^T (upper)
+  float* Linv;      // [kT, kT] the current diagonal block's inverse, row-major
+  int64_t ld;       // np, a multiple of kT
+  int nb;           // np / kT
+  int* fstatus;     // factorization status word
+  unsigned* bar;    // grid barrier: [0] arrivals, [1] generation (zeroed on entry)
+  int* abort;       // set when a wait runs out (zeroed on entry)
   uint64_t wait_ns;
-  int vec;           // rows of four along a tile row are 16-byte aligned (lda, ldx, bases)
-  unsigned* smids;   // [gridDim.x] SM of each CTA
 };
-
-typedef float Tile[kPad];
-
-__device__ __forceinline__ float ld_a(const CholArgs& p, int r, int c) {
-  return (r < p.n && c < p.n) ? __ldcg(p.A + r * p.lda + c) : 0.0f;
-}
-__device__ __forceinline__ float* at_a(const CholArgs& p, int r, int c) { return p.A + r * p.lda + c; }
-__device__ __forceinline__ float* at_x(const CholArgs& p, int r, int c) { return p.X + r * p.ldx + c; }
-
-// acc[i][j] = sum_k P[k][tr+i] * Q[k][tc+j]  (thread owns a 4x4 block)
-__device__ __forceinline__ void tile_product(const Tile* P, const Tile* Q, float (&acc)[4][4]) {
-  const int tr = (threadIdx.x / 16) * 4, tc = (threadIdx.x % 16) * 4;
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
-#pragma unroll 8
-  for (int k = 0; k < kT; ++k) {
-    const float4 a = *reinterpret_cast<const float4*>(&P[k][tr]);
-    const float4 b = *reinterpret_cast<const float4*>(&Q[k][tc]);
-    const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-  }
-}
-
-// Factors the diagonal block k: L_kk into A, Linv_kk into X's diagonal tile.
-//
-// A right-looking sweep over the block's 64 pivots by the whole CTA, with the
-// inverse built in the same sweep (R = I; at pivot j, X_j = R_j / L_jj and
-// R_i -= L_ij X_j for i > j).  Thread t holds row i = t / 4, columns
-// 16 (t % 4) .. 16 (t % 4) + 15 of the block in registers: left of the pivot
-// those are R's entries, right of it the remaining matrix, upper half
-// included.  The upper half makes row j carry, by symmetry, the column under
-// the pivot too, so one broadcast per pivot suffices: the four threads of row
-// j + 1 store their registers to shared memory (R_{j+1,<j+1}, the next pivot,
-// and A_{j+1,>j+1}), one barrier, and every thread reads the pivot, its own
-// row's multiplier and its sixteen columns from there.  With s_i = A_ij / d_j
-// (d_j the pivot), every update is v -= s_i * row_j[c]: the Schur update
-// A_ic -= L_ij L_cj on the right of the pivot and R_ic -= L_ij X_jc on its
-// left; the pivot column itself becomes R_ij = -s_i.  X's rows are scaled by
-// 1 / L_ii at the end.  A pivot that is not positive or not finite sets the
-// status word (a non-finite one takes precedence) and is replaced by 1.
-__device__ void factor_diag(const CholArgs& p, int k, Tile* lout, Tile* xout, Tile* bt) {
-  const int k0 = k * kT;
-  const int kb = min(kT, p.n - k0);
-  const int t = threadIdx.x, i = t >> 2, q = t & 3;
-  float* bbuf = &bt[0][0];  // two 64-float broadcast rows (pivot parity)
-  float v[16];
-#pragma unroll
-  for (int m = 0; m < 16; ++m) {
-    const int c = 16 * q + m;
-    v[m] = (i < kb && c < kb) ? ld_a(p, k0 + i, k0 + c) : (i == c ? 1.0f : 0.0f);
-  }
-  if (i == 0) {
-    float4* d4 = reinterpret_cast<float4*>(bbuf + 16 * q);
-#pragma unroll
-    for (int g = 0; g < 4; ++g) d4[g] = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
-  }
-  __syncthreads();
-  float myrd = 1.0f;
-  bool notpd = false, nonfinite = false;
-#pragma unroll 1
-  for (int j0 = 0; j0 < kT; j0 += 16) {
-    // sixteen pivots per iteration, unrolled so that register indices are constants
-#pragma unroll
-    for (int jj = 0; jj < 16; ++jj) {
-      const int j = j0 + jj;
-      const float* B = bbuf + (j & 1) * kT;
-      float* Bn = bbuf + ((j + 1) & 1) * kT;
-      float d = B[j];
-      const float bi = B[i];
-      float bc[16];
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const float4 w = *reinterpret_cast<const float4*>(B + 16 * q + 4 * g);
-        bc[4 * g] = w.x;
-        bc[4 * g + 1] = w.y;
-        bc[4 * g + 2] = w.z;
-        bc[4 * g + 3] = w.w;
-      }
-      nonfinite |= !isfinite(d);
-      notpd |= !(d > 0.0f);
-      d = (d > 0.0f && d < INFINITY) ? d : 1.0f;
-      const float rd = rsqrtf(d);
-      const float s = bi * rd * rd;
-      if (i > j) {
-#pragma unroll
-        for (int m = 0; m < 16; ++m) v[m] = fmaf(-s, bc[m], v[m]);
-        if (q == (j0 >> 4)) v[jj] = -s;
-      }
-      myrd = i == j ? rd : myrd;
-      if (q == 0 && i >= j) lout[i][j] = (i == j ? d : bi) * rd;
-      if (i == j + 1) {
-        float4* d4 = reinterpret_cast<float4*>(Bn + 16 * q);
-#pragma unroll
-        for (int g = 0; g < 4; ++g) d4[g] = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
-      }
-      __syncthreads();
-    }
-  }
-  if (t == 0 && (nonfinite || notpd)) set_status(p.fstatus, nonfinite ? GPTQ_ERR_NONFINITE : GPTQ_ERR_NOT_PD);
-#pragma unroll
-  for (int m = 0; m < 16; ++m) {
-    const int c = 16 * q + m;
-    xout[i][c] = c < i ? v[m] * myrd : (c == i ? myrd : 0.0f);
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < kT * kT; e += kCholThreads) {
-    const int r = e / kT, c = e % kT;
-    if (r < kb && c < kb) {
-      if (c <= r) *at_a(p, k0 + r, k0 + c) = lout[r][c];
-      *at_x(p, k0 + r, k0 + c) = xout[r][c];
-    }
-  }
-  __syncthreads();
-}
 
 // Time-bounded barrier over the whole (co-resident) grid.
 __device__ bool grid_sync(const CholArgs& p) {
@@ -321,223 +225,431 @@ __device__ bool grid_sync(const CholArgs& p) {
   return ok_s != 0;
 }
 
-// One tile operation of a phase (see the table at the top of this section).
-enum { kOpTrsm = 0, kOpFinalize = 1, kOpUpdate = 2, kOpInverse = 3 };
-struct TileOp {
-  int kind, i0, j0;
-};
-
-__device__ __forceinline__ TileOp op_phase_t(int k, int nb, int t) {
-  const int ntrsm = nb - k - 1;
-  if (t < ntrsm) return {kOpTrsm, (k + 1 + t) * kT, k * kT};
-  return {kOpFinalize, k * kT, (t - ntrsm) * kT};
+__device__ __forceinline__ void give_up(const CholArgs& p) {
+  if (threadIdx.x == 0) {
+    set_status(p.fstatus, GPTQ_ERR_TIMEOUT);
+    atomicExch(p.abort, 1);
+  }
 }
 
-__device__ __forceinline__ TileOp op_phase_u(int k, int nb, int t) {
-  const int m = nb - k - 1;
+__device__ __forceinline__ float* tile_at(float* base, int64_t ld, int i, int j) {
+  return base + static_cast<int64_t>(i) * kT * ld + static_cast<int64_t>(j) * kT;
+}
+
+// One tile operation: C = P Q^T (sub == 0) or C -= P Q^T (sub == 1); all
+// three are 128 x 128 tiles, rows of P and Q along K.
+struct TileOp {
+  const float* P;
+  const float* Q;
+  int64_t ldp, ldq;
+  float* C;
+  int sub;
+};
+
+__device__ TileOp op_phase_t(const CholArgs& p, int k, int t) {
+  const int ntrsm = p.nb - 1 - k;
+  TileOp op;
+  op.Q = p.Linv;
+  op.ldq = kT;
+  op.ldp = p.ld;
+  op.sub = 0;
+  float* c = t < ntrsm ? tile_at(p.A, p.ld, k + 1 + t, k) : tile_at(p.Y, p.ld, t - ntrsm, k);
+  op.P = c;
+  op.C = c;
+  return op;
+}
+
+__device__ TileOp op_phase_u(const CholArgs& p, int k, int t) {
+  const int m = p.nb - 1 - k;
   const int nupd = m * (m + 1) / 2;
-  if (t < nupd) {
+  TileOp op;
+  op.ldp = p.ld;
+  op.ldq = p.ld;
+  op.sub = 1;
+  if (t < nupd) {  // (a, b), b <= a, in row-major order of the lower triangle
     int a = static_cast<int>((sqrtf(8.0f * t + 1.0f) - 1.0f) * 0.5f);
     while ((a + 1) * (a + 2) / 2 <= t) ++a;
     while (a * (a + 1) / 2 > t) --a;
     const int b = t - a * (a + 1) / 2;
-    return {kOpUpdate, (k + 1 + a) * kT, (k + 1 + b) * kT};
-  }
-  const int tt = t - nupd;
-  return {kOpInverse, (k + 1 + tt / (k + 1)) * kT, (tt % (k + 1)) * kT};
-}
-
-// Four consecutive entries (r, c .. c + 3) of A or of X; c % 4 == 0.  Vector
-// loads when p.vec.
-__device__ __forceinline__ float4 ld4(const CholArgs& p, bool from_x, int r, int c) {
-  if (r >= p.n || c >= p.n) return make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  const float* src = from_x ? at_x(p, r, c) : at_a(p, r, c);
-  if (p.vec) return __ldcg(reinterpret_cast<const float4*>(src));
-  return make_float4(__ldcg(src), c + 1 < p.n ? __ldcg(src + 1) : 0.0f, c + 2 < p.n ? __ldcg(src + 2) : 0.0f,
-                     c + 3 < p.n ? __ldcg(src + 3) : 0.0f);
-}
-__device__ __forceinline__ float4 ld4_a(const CholArgs& p, int r, int c) { return ld4(p, false, r, c); }
-__device__ __forceinline__ float4 ld4_x(const CholArgs& p, int r, int c) { return ld4(p, true, r, c); }
-
-__device__ __forceinline__ void st4(const CholArgs& p, bool to_x, int r, int c, float4 v) {
-  if (r >= p.n || c >= p.n) return;
-  float* dst = to_x ? at_x(p, r, c) : at_a(p, r, c);
-  if (p.vec) {
-    *reinterpret_cast<float4*>(dst) = v;
+    const int i = k + 1 + a, j = k + 1 + b;
+    op.P = tile_at(p.A, p.ld, i, k);
+    op.Q = tile_at(p.A, p.ld, j, k);
+    op.C = tile_at(p.A, p.ld, i, j);
   } else {
-    dst[0] = v.x;
-    if (c + 1 < p.n) dst[1] = v.y;
-    if (c + 2 < p.n) dst[2] = v.z;
-    if (c + 3 < p.n) dst[3] = v.w;
+    const int tt = t - nupd;
+    const int i = k + 1 + tt / (k + 1), j = tt % (k + 1);
+    op.P = tile_at(p.Y, p.ld, j, k);
+    op.Q = tile_at(p.A, p.ld, i, k);
+    op.C = tile_at(p.Y, p.ld, j, i);
   }
+  return op;
 }
 
-// Adds v to four consecutive entries (r, c .. c + 3) of A or X in memory (a
-// reduction performed in L2: no read into the SM, nothing to wait for).
-// Each entry receives one such addition per phase, so the result is that of
-// a load, an fp32 addition and a store.
-__device__ __forceinline__ void red4(const CholArgs& p, bool to_x, int r, int c, float4 v) {
-  if (r >= p.n || c >= p.n) return;
-  float* dst = to_x ? at_x(p, r, c) : at_a(p, r, c);
-  if (p.vec) {
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
-                 : "memory");
-  } else {
-    atomicAdd(dst, v.x);
-    if (c + 1 < p.n) atomicAdd(dst + 1, v.y);
-    if (c + 2 < p.n) atomicAdd(dst + 2, v.z);
-    if (c + 3 < p.n) atomicAdd(dst + 3, v.w);
-  }
-}
-
-// Which four entries (row a, columns 4 b4 .. 4 b4 + 3) of a 64 x 64 operand
-// thread t stages in its slot g.  An operand that shared memory keeps
-// transposed uses mapping T: two lanes per row (one 32-byte sector per row and
-// instruction), so that the transposed scalar stores of a warp hit 32
-// distinct banks.  One kept as loaded uses mapping N: 16 lanes along a row,
-// conflict-free vector stores.
-__device__ __forceinline__ void slot_t(int g, int& a, int& b4) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  a = (lane >> 1) + 16 * (warp & 3);
-  b4 = (lane & 1) + 2 * ((warp >> 2) + 2 * g);
-}
-__device__ __forceinline__ void slot_n(int g, int& a, int& b4) {
-  const int idx = g * kCholThreads + threadIdx.x;
-  a = idx >> 4;
-  b4 = idx & 15;
-}
-
-// Registers holding one tile operation's operands between their loads and
-// their use.
-struct Staged {
+// The registers holding one chunk of both operands: thread t loads rows
+// t / 8 + 32 g (g < 4), 16 bytes at column 4 (t % 8) of the chunk.
+struct Chunk {
   float4 p[4], q[4];
 };
 
-__device__ __forceinline__ bool q_natural(const TileOp& op) { return op.kind == kOpFinalize || op.kind == kOpInverse; }
-
-// The first operand of an operation: A_ik / L_ik (row block i of panel k) for
-// trsm, update and inverse, Linv_kk for finalize.  Consecutive operations
-// with the same key share it, so it is loaded and staged once.
-__device__ __forceinline__ int p_key(const TileOp& op) { return op.kind == kOpFinalize ? -2 : op.i0; }
-
-__device__ __forceinline__ void fetch_op(const CholArgs& p, const TileOp& op, int k0, Staged& st, bool need_p) {
+__device__ __forceinline__ void load_chunk(const TileOp& op, int c, Chunk& ch) {
+  const int cc = threadIdx.x & 7, r0 = threadIdx.x >> 3;
 #pragma unroll
   for (int g = 0; g < 4; ++g) {
-    int a, b4, an, bn4;
-    slot_t(g, a, b4);
-    slot_n(g, an, bn4);
-    const int b = 4 * b4;
-    if (!need_p) {  // the second operand only (as in the cases below)
-      switch (op.kind) {
-        case kOpTrsm:
-          st.q[g] = ld4_x(p, k0 + a, k0 + b);
-          break;
-        case kOpUpdate:
-          st.q[g] = ld4_a(p, op.j0 + a, k0 + b);
-          break;
-        default:
-          st.q[g] = ld4_x(p, k0 + an, op.j0 + 4 * bn4);
-          break;
-      }
-      continue;
-    }
-    switch (op.kind) {
-      case kOpTrsm:      // A_ik * Linv_kk^T
-        st.p[g] = ld4_a(p, op.i0 + a, k0 + b);
-        st.q[g] = ld4_x(p, k0 + a, k0 + b);
-        break;
-      case kOpFinalize:  // Linv_kk * R_kj
-        st.p[g] = ld4_x(p, k0 + a, k0 + b);
-        st.q[g] = ld4_x(p, k0 + an, op.j0 + 4 * bn4);
-        break;
-      case kOpUpdate:    // A_ij - L_ik L_jk^T
-        st.p[g] = ld4_a(p, op.i0 + a, k0 + b);
-        st.q[g] = ld4_a(p, op.j0 + a, k0 + b);
-        break;
-      default:           // R_ij - L_ik X_kj
-        st.p[g] = ld4_a(p, op.i0 + a, k0 + b);
-        st.q[g] = ld4_x(p, k0 + an, op.j0 + 4 * bn4);
-        break;
-    }
+    const int r = r0 + 32 * g;
+    ch.p[g] = __ldcg(reinterpret_cast<const float4*>(op.P + r * op.ldp + c * kCk + 4 * cc));
+    ch.q[g] = __ldcg(reinterpret_cast<const float4*>(op.Q + r * op.ldq + c * kCk + 4 * cc));
   }
 }
 
-// P is always used as P[r][k]; Q as Q[c][k] (transposed load) for the
-// Cholesky operations and as Q[k][c] (natural load) for the inverse ones.
-__device__ __forceinline__ void commit_op(const TileOp& op, const Staged& st, Tile* sp, Tile* sq, bool write_p) {
-  const bool qn = q_natural(op);
+__device__ __forceinline__ float tf32_hi(float x) { return __uint_as_float(__float_as_uint(x) & 0xffffe000u); }
+
+__device__ __forceinline__ void put_split(uint8_t* hi, uint8_t* lo, uint32_t off, float4 v) {
+  const float4 h = make_float4(tf32_hi(v.x), tf32_hi(v.y), tf32_hi(v.z), tf32_hi(v.w));
+  *reinterpret_cast<float4*>(hi + off) = h;
+  *reinterpret_cast<float4*>(lo + off) = make_float4(v.x - h.x, v.y - h.y, v.z - h.z, v.w - h.w);
+}
+
+// Row r of a 128 x 32 fp32 operand chunk is one 128-byte row of the buffer
+// whose 16-byte pieces are permuted by XOR with (r mod 8): the layout a TMA
+// load with 128-byte swizzle writes, read by the MMA descriptors below.
+__device__ __forceinline__ void store_chunk(uint8_t* stage, const Chunk& ch) {
+  const int cc = threadIdx.x & 7, r0 = threadIdx.x >> 3;
 #pragma unroll
   for (int g = 0; g < 4; ++g) {
-    int a, b4;
-    slot_t(g, a, b4);
-    const int b = 4 * b4;
-    if (write_p) {
-      sp[b + 0][a] = st.p[g].x;
-      sp[b + 1][a] = st.p[g].y;
-      sp[b + 2][a] = st.p[g].z;
-      sp[b + 3][a] = st.p[g].w;
-    }
-    if (qn) {
-      int an, bn4;
-      slot_n(g, an, bn4);
-      *reinterpret_cast<float4*>(&sq[an][4 * bn4]) = st.q[g];
-    } else {
-      sq[b + 0][a] = st.q[g].x;
-      sq[b + 1][a] = st.q[g].y;
-      sq[b + 2][a] = st.q[g].z;
-      sq[b + 3][a] = st.q[g].w;
-    }
+    const int r = r0 + 32 * g;
+    const uint32_t off = static_cast<uint32_t>(r * 128 + ((cc ^ (r & 7)) << 4));
+    put_split(stage, stage + kBufBytes, off, ch.p[g]);
+    put_split(stage + 2 * kBufBytes, stage + 3 * kBufBytes, off, ch.q[g]);
   }
 }
 
-// Writes the product (trsm, finalize) or subtracts it in place (update,
-// inverse: an L2 reduction, so the old values never travel to the SM).
-__device__ __forceinline__ void finish_op(const CholArgs& p, const TileOp& op, int k0, const float (&acc)[4][4]) {
-  const int tr = (threadIdx.x / 16) * 4, tc = (threadIdx.x % 16) * 4;
-  const bool to_x = op.kind == kOpFinalize || op.kind == kOpInverse;
-  const bool subtract = op.kind == kOpUpdate || op.kind == kOpInverse;
-  const int r0 = op.kind == kOpFinalize ? k0 : op.i0;
-  const int c0 = op.kind == kOpTrsm ? k0 : op.j0;
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// The three tf32 products of one staged chunk (4 K-steps of 8) into d_tmem.
+__device__ __forceinline__ void issue_chunk(const uint8_t* stage, uint32_t d_tmem, bool first) {
+  const uint32_t idesc = instr_desc(2u, 0u, 0u, kT, kT);  // tf32, both operands K-major, 128 x 128
+  const uint32_t ph = smem_u32(stage), pl = ph + kBufBytes, qh = pl + kBufBytes, ql = qh + kBufBytes;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    if (subtract)
-      red4(p, to_x, r0 + tr + i, c0 + tc, make_float4(-acc[i][0], -acc[i][1], -acc[i][2], -acc[i][3]));
-    else
-      st4(p, to_x, r0 + tr + i, c0 + tc, make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]));
+  for (int kk = 0; kk < kCk / 8; ++kk) {
+    // K-major: the next 8 columns of K are 32 bytes further along each row
+    const uint64_t dph = smem_desc_sw128(ph + kk * 32, 16, 1024);
+    const uint64_t dpl = smem_desc_sw128(pl + kk * 32, 16, 1024);
+    const uint64_t dqh = smem_desc_sw128(qh + kk * 32, 16, 1024);
+    const uint64_t dql = smem_desc_sw128(ql + kk * 32, 16, 1024);
+    mma_tf32(d_tmem, dph, dqh, idesc, (first && kk == 0) ? 0u : 1u);
+    mma_tf32(d_tmem, dph, dql, idesc, 1u);
+    mma_tf32(d_tmem, dpl, dqh, idesc, 1u);
   }
 }
 
-// Runs the tile operations [lo, hi) of one phase.  Operations are numbered
-// row block by row block, so consecutive ones mostly share their first
-// operand, which then stays in shared memory.  The operands of the next
-// operation are loaded into registers while the current one is multiplied,
-// so L2 latency overlaps the FMAs.
+__device__ __forceinline__ void red4(float* dst, float4 v) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+               : "memory");
+}
+
+// The accumulator into the output tile: warp w reads lanes 32 (w % 4) .. + 31
+// (tile rows) and columns 64 (w / 4) .. + 63, and stores them (or subtracts
+// them as L2 reductions, so the old values never travel to the SM).
+__device__ __forceinline__ void write_tile(const TileOp& op, int64_t ld, uint32_t acc) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int quad = warp & 3, half = warp >> 2;
+  float* row = op.C + static_cast<int64_t>(32 * quad + lane) * ld;
+#pragma unroll
+  for (int x = 0; x < 2; ++x) {
+    const int c0 = 64 * half + 32 * x;
+    uint32_t v[32];
+    tmem_ld_32x32b_x32(acc + (static_cast<uint32_t>(32 * quad) << 16) + static_cast<uint32_t>(c0), v);
+    tmem_ld_wait();
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float4 f = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                   __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+      if (op.sub)
+        red4(row + c0 + 4 * q, make_float4(-f.x, -f.y, -f.z, -f.w));
+      else
+        *reinterpret_cast<float4*>(row + c0 + 4 * q) = f;
+    }
+  }
+}
+
+// Per-CTA pipeline state (identical in every thread).
+struct Pipe {
+  uint8_t* ring;         // kStages stages of kStageBytes, 1024-byte aligned
+  uint64_t* stage_free;  // [kStages]: completes when the MMAs reading a stage are done
+  uint64_t* acc_full;    // [2]: completes when an accumulator's products are done
+  uint64_t* drain;
+  uint32_t tmem;         // base of the two accumulators
+  uint32_t chunks;       // chunks staged so far (all phases)
+  uint32_t ops;          // operations issued so far
+};
+
+// Waits for operation number o's products and writes its tile.
+__device__ bool finish_op(const CholArgs& p, const Pipe& pp, const TileOp& op, uint32_t o) {
+  const bool ok = mbar_wait(pp.acc_full + (o & 1u), (o >> 1) & 1u, p.wait_ns);
+  if (!__syncthreads_and(ok)) {
+    give_up(p);
+    return false;
+  }
+  tc_fence_after();
+  write_tile(op, p.ld, pp.tmem + (o & 1u) * kT);
+  tc_fence_before();
+  return true;
+}
+
+// Runs operations [lo, hi) of a phase.  Returns false if a wait ran out.
+// On return every product this CTA issued is done.
 template <bool kPhaseU>
-__device__ void run_phase(const CholArgs& p, int k, int lo, int hi, Tile* s0, Tile* s1) {
-  if (lo >= hi) return;
-  const int nb = p.nblk, k0 = k * kT;
-  Staged st;
-  TileOp cur = kPhaseU ? op_phase_u(k, nb, lo) : op_phase_t(k, nb, lo);
-  fetch_op(p, cur, k0, st, true);
-  bool write_p = true;
+__device__ bool run_ops(const CholArgs& p, Pipe& pp, int k, int lo, int hi) {
+  if (lo >= hi) return true;
+  Chunk ch;
+  TileOp cur = kPhaseU ? op_phase_u(p, k, lo) : op_phase_t(p, k, lo);
+  TileOp prev = cur;
+  load_chunk(cur, 0, ch);
   for (int t = lo; t < hi; ++t) {
-    commit_op(cur, st, s0, s1, write_p);
-    __syncthreads();
-    TileOp nxt = cur;
-    bool next_p = false;
-    if (t + 1 < hi) {
-      nxt = kPhaseU ? op_phase_u(k, nb, t + 1) : op_phase_t(k, nb, t + 1);
-      next_p = p_key(nxt) != p_key(cur);
-      fetch_op(p, nxt, k0, st, next_p);
+    const bool more = t + 1 < hi;
+    const TileOp nxt = more ? (kPhaseU ? op_phase_u(p, k, t + 1) : op_phase_t(p, k, t + 1)) : cur;
+    const uint32_t buf = pp.ops & 1u;
+#pragma unroll 1
+    for (int c = 0; c < kChunks; ++c) {
+      const uint32_t s = pp.chunks % kStages;
+      uint8_t* stage = pp.ring + s * kStageBytes;
+      bool ok = true;
+      if (pp.chunks >= kStages)  // the products that read this stage two chunks ago
+        ok = mbar_wait(pp.stage_free + s, ((pp.chunks - kStages) / kStages) & 1u, p.wait_ns);
+      if (ok) store_chunk(stage, ch);
+      if (c + 1 < kChunks)
+        load_chunk(cur, c + 1, ch);
+      else if (more)
+        load_chunk(nxt, 0, ch);
+      fence_async_smem();
+      if (!__syncthreads_and(ok)) {
+        give_up(p);
+        return false;
+      }
+      if (threadIdx.x == 0) {
+        tc_fence_after();
+        issue_chunk(stage, pp.tmem + buf * kT, c == 0);
+        mma_commit(pp.stage_free + s);
+        if (c + 1 == kChunks) mma_commit(pp.acc_full + buf);
+      }
+      ++pp.chunks;
     }
-    float acc[4][4];
-    tile_product(s0, s1, acc);
-    finish_op(p, cur, k0, acc);
-    __syncthreads();
+    if (t > lo && !finish_op(p, pp, prev, pp.ops - 1)) return false;
+    prev = cur;
     cur = nxt;
-    write_p = next_p;
+    ++pp.ops;
   }
-  __threadfence();  // this CTA's reductions are performed before its later reads
+  return finish_op(p, pp, prev, pp.ops - 1);
+}
+
+// Right-looking Cholesky of a 16 x 16 block held by one warp: lane l holds
+// row l / 2, columns 8 (l % 2) .. + 7 in v (only the lower half is read).
+// On return v holds L's lower half and rdiag[j] = 1 / L_jj.  A pivot that is
+// not positive or not finite raises a flag and is replaced by 1.
+__device__ __forceinline__ void chol16(float (&v)[8], float* rdiag, bool& nonfinite, bool& notpd) {
+  const int lane = threadIdx.x & 31, r = lane >> 1, h = lane & 1;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int jh = j >> 3, jq = j & 7;
+    float d = __shfl_sync(0xffffffffu, v[jq], 2 * j + jh);        // A_jj
+    const float mine = __shfl_sync(0xffffffffu, v[jq], 2 * r + jh);  // A_rj
+    float col[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) col[q] = __shfl_sync(0xffffffffu, v[jq], 2 * (8 * h + q) + jh);  // A_cj
+    nonfinite |= !isfinite(d);
+    notpd |= !(d > 0.0f);
+    d = (d > 0.0f && d < INFINITY) ? d : 1.0f;
+    const float rs = rsqrtf(d);
+    const float lr = mine * rs;  // L_rj
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int c = 8 * h + q;
+      if (c > j && c <= r) v[q] = fmaf(-lr, col[q] * rs, v[q]);
+    }
+    if (h == jh) v[jq] = r > j ? lr : (r == j ? d * rs : v[jq]);
+    if (lane == 0) rdiag[j] = rs;
+  }
+}
+
+// x <- L_ss^-1 x for the sub-block's factor (lower half of S at (b0, b0))
+// and its reciprocal diagonal: the forward substitution both halves of
+// phase A below use (for rows of the panel x holds S_i,s, for columns of the
+// inverse R_s,j).
+__device__ __forceinline__ void solve16(float (&x)[16], const float* S, const float* rd, int b0) {
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    x[c] *= rd[b0 + c];
+#pragma unroll
+    for (int c2 = c + 1; c2 < 16; ++c2) x[c2] = fmaf(-x[c], S[(b0 + c2) * kSP + b0 + c], x[c2]);
+  }
+}
+
+// Factors the diagonal block k (by one CTA): Linv_kk into p.Linv (row-major)
+// and Y_kk = Linv_kk^T into Y's diagonal tile.
+//
+// In 16-wide sub-panels s of the block S (its lower half), with R = I beside it:
+//   warp 0   Cholesky of the sub-panel's 16 x 16 diagonal block (chol16)
+//   phase A  rows i below: L_i,s = S_i,s L_ss^-T, one thread per row, into
+//            the panel buffer Pn (transposed); columns j < end of the
+//            sub-panel: X_s,j = L_ss^-1 R_s,j, one thread per column, in place
+//   phase B  S_ic -= L_i,s L_c,s^T (c <= i below the sub-panel) and
+//            R_ij -= L_i,s X_s,j (i below, j < end of the sub-panel) in 4 x 4
+//            blocks; warp 0 first updates the next diagonal 16 x 16 block and
+//            factors it (the sweep's critical path).
+// A pivot that is not positive or not finite sets the status word (a
+// non-finite one takes precedence) and is replaced by 1.
+__device__ void factor_block(const CholArgs& p, int k, float* fs) {
+  float* S = fs;                // [kT][kSP]
+  float* XR = S + kT * kSP;     // [kT][kSP]: R, then X = L^-1 (lower)
+  float* Pn = XR + kT * kSP;    // [kSub][kT]: the current sub-panel of L, transposed
+  float* rd = Pn + kSub * kT;   // [kT]: 1 / L_jj
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const float* Akk = tile_at(p.A, p.ld, k, k);
+  for (int e = t; e < kT * (kT / 4); e += kCholThreads) {
+    const int r = e >> 5, c = 4 * (e & 31);
+    *reinterpret_cast<float4*>(S + r * kSP + c) = __ldcg(reinterpret_cast<const float4*>(Akk + r * p.ld + c));
+    *reinterpret_cast<float4*>(XR + r * kSP + c) =
+        make_float4(r == c ? 1.0f : 0.0f, r == c + 1 ? 1.0f : 0.0f, r == c + 2 ? 1.0f : 0.0f, r == c + 3 ? 1.0f : 0.0f);
+  }
+  __syncthreads();
+  bool nonfinite = false, notpd = false;
+  if (warp == 0) {
+    const int r = lane >> 1, h = lane & 1;
+    float v[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) v[q] = S[r * kSP + 8 * h + q];
+    chol16(v, rd, nonfinite, notpd);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) S[r * kSP + 8 * h + q] = v[q];
+  }
+  __syncthreads();
+#pragma unroll 1
+  for (int s = 0; s < kT / kSub; ++s) {
+    const int b0 = s * kSub, e = b0 + kSub;
+    // phase A
+    if (t < kT - e) {
+      const int i = e + t;
+      float x[16];
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const float4 w = *reinterpret_cast<const float4*>(S + i * kSP + b0 + 4 * g);
+        x[4 * g] = w.x;
+        x[4 * g + 1] = w.y;
+        x[4 * g + 2] = w.z;
+        x[4 * g + 3] = w.w;
+      }
+      solve16(x, S, rd, b0);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) Pn[c * kT + i] = x[c];
+    } else if (t >= kT && t - kT < e) {
+      const int j = t - kT;
+      float x[16];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) x[c] = XR[(b0 + c) * kSP + j];
+      solve16(x, S, rd, b0);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) XR[(b0 + c) * kSP + j] = x[c];
+    }
+    __syncthreads();
+    if (e == kT) break;
+    // phase B
+    if (warp == 0) {
+      const int r = lane >> 1, h = lane & 1, i = e + r, c0 = e + 8 * h;
+      float v[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = S[i * kSP + c0 + q];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const float li = Pn[q * kT + i];
+        const float4 a = *reinterpret_cast<const float4*>(Pn + q * kT + c0);
+        const float4 b = *reinterpret_cast<const float4*>(Pn + q * kT + c0 + 4);
+        v[0] = fmaf(-li, a.x, v[0]);
+        v[1] = fmaf(-li, a.y, v[1]);
+        v[2] = fmaf(-li, a.z, v[2]);
+        v[3] = fmaf(-li, a.w, v[3]);
+        v[4] = fmaf(-li, b.x, v[4]);
+        v[5] = fmaf(-li, b.y, v[5]);
+        v[6] = fmaf(-li, b.z, v[6]);
+        v[7] = fmaf(-li, b.w, v[7]);
+      }
+      chol16(v, rd + e, nonfinite, notpd);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) S[i * kSP + c0 + q] = v[q];
+    } else {
+      const int M4 = (kT - e) / 4, E4 = e / 4;
+      const int ntr = M4 * (M4 + 1) / 2 - 10;  // lower 4 x 4 blocks outside warp 0's 16 x 16 block
+      const int total = ntr + M4 * E4;
+      for (int w = t - 32; w < total; w += kCholThreads - 32) {
+        float acc[4][4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[r][c] = 0.0f;
+        float* dst;
+        if (w < ntr) {
+          const int idx = w + 10;
+          int a = static_cast<int>((sqrtf(8.0f * idx + 1.0f) - 1.0f) * 0.5f);
+          while ((a + 1) * (a + 2) / 2 <= idx) ++a;
+          while (a * (a + 1) / 2 > idx) --a;
+          const int bb = idx - a * (a + 1) / 2;
+          const int i0 = e + 4 * a, c0 = e + 4 * bb;
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            const float4 li = *reinterpret_cast<const float4*>(Pn + q * kT + i0);
+            const float4 lc = *reinterpret_cast<const float4*>(Pn + q * kT + c0);
+            const float lv[4] = {li.x, li.y, li.z, li.w}, cv[4] = {lc.x, lc.y, lc.z, lc.w};
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+              for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(lv[r], cv[c], acc[r][c]);
+          }
+          dst = S + i0 * kSP + c0;
+        } else {
+          const int w2 = w - ntr;
+          const int i0 = e + 4 * (w2 / E4), j0 = 4 * (w2 % E4);
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            const float4 li = *reinterpret_cast<const float4*>(Pn + q * kT + i0);
+            const float4 xq = *reinterpret_cast<const float4*>(XR + (b0 + q) * kSP + j0);
+            const float lv[4] = {li.x, li.y, li.z, li.w}, xv[4] = {xq.x, xq.y, xq.z, xq.w};
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+              for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(lv[r], xv[c], acc[r][c]);
+          }
+          dst = XR + i0 * kSP + j0;
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          float4 o = *reinterpret_cast<float4*>(dst + r * kSP);
+          o.x -= acc[r][0];
+          o.y -= acc[r][1];
+          o.z -= acc[r][2];
+          o.w -= acc[r][3];
+          *reinterpret_cast<float4*>(dst + r * kSP) = o;
+        }
+      }
+    }
+    __syncthreads();
+  }
+  if (warp == 0) {
+    nonfinite = __any_sync(0xffffffffu, nonfinite);
+    notpd = __any_sync(0xffffffffu, notpd);
+    if (lane == 0 && (nonfinite || notpd)) set_status(p.fstatus, nonfinite ? GPTQ_ERR_NONFINITE : GPTQ_ERR_NOT_PD);
+  }
+  // Linv (row-major, zeros above the diagonal) and Y_kk = Linv^T
+  float* Ykk = tile_at(p.Y, p.ld, k, k);
+  for (int e = t; e < kT * (kT / 4); e += kCholThreads) {
+    const int r = e >> 5, c = 4 * (e & 31);
+    const float4 x = *reinterpret_cast<const float4*>(XR + r * kSP + c);
+    *reinterpret_cast<float4*>(p.Linv + r * kT + c) =
+        make_float4(c <= r ? x.x : 0.0f, c + 1 <= r ? x.y : 0.0f, c + 2 <= r ? x.z : 0.0f, c + 3 <= r ? x.w : 0.0f);
+    const int ry = e & (kT - 1), cy = 4 * (e >> 7);  // Y_kk[ry][cy + u] = X[cy + u][ry]
+    *reinterpret_cast<float4*>(Ykk + ry * p.ld + cy) =
+        make_float4(cy >= ry ? XR[cy * kSP + ry] : 0.0f, cy + 1 >= ry ? XR[(cy + 1) * kSP + ry] : 0.0f,
+                    cy + 2 >= ry ? XR[(cy + 2) * kSP + ry] : 0.0f, cy + 3 >= ry ? XR[(cy + 3) * kSP + ry] : 0.0f);
+  }
+  __threadfence();
   __syncthreads();
 }
 
@@ -547,137 +659,127 @@ __device__ __forceinline__ void share(int total, int w, int workers, int& lo, in
   hi = static_cast<int>((static_cast<int64_t>(total) * (w + 1)) / workers);
 }
 
-__device__ __forceinline__ unsigned sm_id() {
-  unsigned r;
-  asm volatile("mov.u32 %0, %%smid;" : "=r"(r));
-  return r;
-}
-
-__global__ void __launch_bounds__(kCholThreads, 2) chol_inv_kernel(CholArgs p) {
-  extern __shared__ __align__(16) float chol_smem[];
-  __shared__ int sib_s;
-  Tile* s0 = reinterpret_cast<Tile*>(chol_smem);
-  Tile* s1 = s0 + kT;
-  Tile* s2 = s1 + kT;
-  const int nb = p.nblk;
-  const int G = static_cast<int>(gridDim.x), b = static_cast<int>(blockIdx.x);
-  // Every CTA records its SM; the CTA that shares CTA 0's SM (if any) takes no
-  // tile operations, so the diagonal factorizations (the kernel's critical
-  // path, run by CTA 0) have their SM to themselves.
-  if (threadIdx.x == 0) p.smids[b] = sm_id();
-  if (threadIdx.x == 0) sib_s = -1;
-  if (b == 0) factor_diag(p, 0, s0, s1, s2);
-  if (!grid_sync(p)) return;
-  {
-    const unsigned sm0 = __ldcg(p.smids);
-    for (int c = 1 + threadIdx.x; c < G; c += blockDim.x)
-      if (__ldcg(p.smids + c) == sm0) atomicMax(&sib_s, c);
-    __syncthreads();
+__global__ void __launch_bounds__(kCholThreads, 1) chol_tc_kernel(CholArgs p) {
+  extern __shared__ uint8_t chol_smem_raw[];
+  uint8_t* region =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(chol_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(region + kRegionBytes);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 6);
+  const int warp = threadIdx.x >> 5;
+  Pipe pp;
+  pp.ring = region;
+  pp.stage_free = bars;
+  pp.acc_full = bars + 2;
+  pp.drain = bars + 4;
+  pp.chunks = 0;
+  pp.ops = 0;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 5; ++i) mbar_init(bars + i, 1);
+    fence_barrier_init();
   }
-  const int sib = sib_s;
-  const bool idle = (b == sib);
-  const int pidx = b - ((sib >= 0 && b > sib) ? 1 : 0);  // index among the CTAs that work
-  const int PT = G - (sib >= 0 ? 1 : 0);
-  const int W = PT - 1;                                    // workers besides CTA 0
-  for (int k = 0; k < nb; ++k) {
-    // phase T(k): trsm of panel k and row k of the inverse
-    if (!idle) {
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kCholTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  pp.tmem = *tmem_slot;
+  float* fs = reinterpret_cast<float*>(region);  // the diagonal factor's matrices (between products)
+  const int G = static_cast<int>(gridDim.x), b = static_cast<int>(blockIdx.x), nb = p.nb;
+
+  if (b == 0) factor_block(p, 0, fs);
+  bool live = grid_sync(p);
+  for (int k = 0; k < nb && live; ++k) {
+    {  // phase T(k)
       int lo, hi;
-      share(nb - 1, pidx, PT, lo, hi);
-      run_phase<false>(p, k, lo, hi, s0, s1);
+      share(nb - 1, b, G, lo, hi);
+      live = run_ops<false>(p, pp, k, lo, hi);
+      __threadfence();
+      if (live) live = grid_sync(p);
     }
-    if (!grid_sync(p)) return;
-    // phase U(k): CTA 0 updates tile (k+1, k+1) and then factors it; the
-    // other CTAs share the remaining updates, so the factorization is the only
-    // extra work on the critical path.  The factorization runs outside the
-    // pipelined loop, where no prefetched operands are live.
-    const int m = nb - k - 1;
-    const int total = m * (m + 1) / 2 + m * (k + 1);
-    if (W == 0) {
-      if (b == 0) run_phase<true>(p, k, 0, total, s0, s1);
-    } else if (b == 0) {
-      run_phase<true>(p, k, 0, total > 0 ? 1 : 0, s0, s1);
-    } else if (!idle && total > 1) {
-      int lo, hi;
-      share(total - 1, pidx - 1, W, lo, hi);
-      run_phase<true>(p, k, 1 + lo, 1 + hi, s0, s1);
+    if (!live) break;
+    {  // phase U(k): CTA 0 updates tile (k+1, k+1) and factors it while the others share the rest
+      const int m = nb - 1 - k;
+      const int total = m * (m + 1) / 2 + m * (k + 1);
+      if (G == 1) {
+        live = run_ops<true>(p, pp, k, 0, total);
+        if (live && m > 0) factor_block(p, k + 1, fs);
+      } else if (b == 0) {
+        live = run_ops<true>(p, pp, k, 0, total > 0 ? 1 : 0);
+        __threadfence();
+        __syncthreads();
+        if (live && m > 0) factor_block(p, k + 1, fs);
+      } else if (total > 1) {
+        int lo, hi;
+        share(total - 1, b - 1, G - 1, lo, hi);
+        live = run_ops<true>(p, pp, k, 1 + lo, 1 + hi);
+      }
+      __threadfence();
+      if (live) live = grid_sync(p);
     }
-    if (b == 0 && m > 0) factor_diag(p, k + 1, s0, s1, s2);
-    if (!grid_sync(p)) return;
+  }
+  // every exit: this CTA's tensor-core work done, then its tensor memory released
+  if (threadIdx.x == 0) {
+    mma_commit(pp.drain);
+    if (!mbar_wait(pp.drain, 0u, kDrainNs)) set_status(p.fstatus, GPTQ_ERR_TIMEOUT);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(pp.tmem, kCholTmemCols);
   }
 }
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-constexpr int kNB = 1024;  // diagonal block of the blocked factorization
-// From this order on, 1024-wide blocks joined by tensor-core GEMMs.  Below it
-// the single cooperative kernel is faster (2.9 vs 4.4 ms at 4096: the blocked
-// form runs the same 64-wide panel chain plus the GEMM launches) and more
-// accurate (U^T U H' v = v to ~7e-7 vs ~4e-6: the tensor-core accumulation
-// of each 128-long K chunk rounds like truncation).  At 8192 the two take the
-// same time; at 11008 the blocked form is 1.15x faster, and its advantage
-// grows with n (its O(n^3) part runs on the tensor cores).
-constexpr int kBlockedMinN = 8192;
+inline int64_t padded_order(int n) { return ceil_div(n, kT) * kT; }
 
 struct PrepLayout {
-  size_t a, key, dead, lambda, bar, perm, ahi, alo, bhi, blo, panel, total;
+  size_t a, y, linv, key, dead, lambda, bar, perm, total;
 };
 
 PrepLayout prep_layout(int n) {
   PrepLayout l{};
-  const size_t nn = static_cast<size_t>(n) * n;
+  const int64_t np = padded_order(n);
+  const size_t nn = static_cast<size_t>(np) * static_cast<size_t>(np) * sizeof(float);
   size_t off = 0;
   l.a = off;
-  off += align256(nn * sizeof(float));
+  off += align256(nn);
+  l.y = off;
+  off += align256(nn);
+  l.linv = off;
+  off += align256(static_cast<size_t>(kT) * kT * sizeof(float));
   l.key = off;
   off += align256(static_cast<size_t>(n) * sizeof(double));
   l.dead = off;
   off += align256(static_cast<size_t>(n));
   l.lambda = off;
   off += 256;
-  l.bar = off;  // barrier words and the abort flag, then one SM id per CTA
-  off += 256 + align256(kMaxCholCtas * sizeof(unsigned));
+  l.bar = off;  // barrier words and the abort flag
+  off += 256;
   l.perm = off;
   off += align256(static_cast<size_t>(n) * sizeof(int32_t));
-  // blocked factorization (n > kNB): tf32 halves of the GEMM operands and the
-  // panel L_>K,K, each at most n x kNB
-  const size_t blk = n >= kBlockedMinN ? align256(static_cast<size_t>(n) * kNB * sizeof(float)) : 0;
-  l.ahi = off;
-  off += blk;
-  l.alo = off;
-  off += blk;
-  l.bhi = off;
-  off += blk;
-  l.blo = off;
-  off += blk;
-  l.panel = off;
-  off += blk;
   l.total = off;
   return l;
 }
 
 int chol_grid(const DeviceInfo* info) {
-  static std::atomic<int> blocks_per_sm[64] = {};  // per device, shared by host threads
-  if (blocks_per_sm[info->device] == 0) {
+  static std::atomic<int> fits[64] = {};  // per device, shared by host threads: 1 = a CTA fits on an SM
+  if (fits[info->device] == 0) {
     int b = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, chol_inv_kernel, kCholThreads, kCholSmem) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, chol_tc_kernel, kCholThreads, kCholSmem) != cudaSuccess ||
         b < 1)
       return 0;
-    blocks_per_sm[info->device] = std::min(b, 2);
+    fits[info->device] = 1;
   }
-  return std::min(kMaxCholCtas, blocks_per_sm[info->device] * info->sm_count);
+  return std::min(kMaxCholCtas, info->sm_count);  // one CTA per SM (its shared memory and tensor memory)
 }
 
 }  // namespace
 
 size_t prepare_workspace_size(int n) { return n > 0 ? prep_layout(n).total : 0; }
-
-gptq_status split_rows_tf32(const float* src, int64_t lds, int rows, int cols, int kpad, float sign, float* hi,
-                            float* lo, cudaStream_t st);
-gptq_status split_cols_tf32(const float* src, int64_t lds, int rows, int cols, int kpad, float sign, float* hi,
-                            float* lo, cudaStream_t st);
-gptq_status gemm_nt_tc(float* C, int64_t ldc, int M, int N, int kpad, const float* A_hi, const float* A_lo,
-                       const float* B_hi, const float* B_lo, cudaStream_t st);
 
 gptq_status prepare_hinv(const float* H, const double* hdiag, int n, float damp, int act_order, int32_t* perm_out,
                          uint8_t* dead_out, float* U, void* ws, size_t ws_bytes, cudaStream_t st) {
@@ -686,7 +788,9 @@ gptq_status prepare_hinv(const float* H, const double* hdiag, int n, float damp,
   const PrepLayout l = prep_layout(n);
   if (ws_bytes < l.total) return GPTQ_ERR_INVALID_ARG;
   uint8_t* w = static_cast<uint8_t*>(ws);
+  const int64_t np = padded_order(n);
   float* A = reinterpret_cast<float*>(w + l.a);
+  float* Y = reinterpret_cast<float*>(w + l.y);
   double* key = reinterpret_cast<double*>(w + l.key);
   uint8_t* dead = w + l.dead;
   double* lambda = reinterpret_cast<double*>(w + l.lambda);
@@ -696,7 +800,7 @@ gptq_status prepare_hinv(const float* H, const double* hdiag, int n, float damp,
 
   static std::atomic<bool> attr_set[64] = {};  // per device, shared by host threads
   if (!attr_set[info->device]) {
-    if (cudaFuncSetAttribute(chol_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(chol_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kCholSmem)) != cudaSuccess)
       return GPTQ_ERR_CUDA;
     attr_set[info->device] = true;
@@ -713,78 +817,30 @@ gptq_status prepare_hinv(const float* H, const double* hdiag, int n, float damp,
     launch(identity_perm_kernel, static_cast<unsigned>(ceil_div(n, 256)), 256, 0, st, perm, n);
   if (dead_out != nullptr && cudaMemcpyAsync(dead_out, dead, n, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
     return GPTQ_ERR_CUDA;
-  launch(gather_reversed_kernel, dim3(static_cast<unsigned>(ceil_div(n, 256)), n), 256, 0, st, H, perm, dead, lambda,
-         n, A);
-  if (cudaMemsetAsync(U, 0, static_cast<size_t>(n) * n * sizeof(float), st) != cudaSuccess) return GPTQ_ERR_CUDA;
+  launch(gather_reversed_kernel, dim3(static_cast<unsigned>(ceil_div(np, 256)), static_cast<unsigned>(std::min<int64_t>(np, 65535))),
+         256, 0, st, H, perm, dead, lambda, n, np, A);
+  if (cudaMemsetAsync(Y, 0, static_cast<size_t>(np) * static_cast<size_t>(np) * sizeof(float), st) != cudaSuccess)
+    return GPTQ_ERR_CUDA;
   if (launch_status() != GPTQ_OK) return GPTQ_ERR_CUDA;
 
-  // The diagonal block [k0, k0 + kb) through the cooperative kernel; X = U
-  // (unrotated until the end).
-  auto factor_block = [&](int k0, int kb) -> gptq_status {
-    if (cudaMemsetAsync(bar, 0, 256, st) != cudaSuccess) return GPTQ_ERR_CUDA;
-    CholArgs ca;
-    ca.A = A + static_cast<int64_t>(k0) * n + k0;
-    ca.X = U + static_cast<int64_t>(k0) * n + k0;
-    ca.lda = n;
-    ca.ldx = n;
-    ca.n = kb;
-    ca.nblk = static_cast<int>(ceil_div(kb, kT));
-    ca.fstatus = fstatus;
-    ca.bar = bar;
-    ca.abort = reinterpret_cast<int*>(bar + 2);
-    ca.smids = bar + 64;
-    ca.wait_ns = wait_limit_ns();
-    ca.vec = (n % 4 == 0) ? 1 : 0;
-    void* args[] = {&ca};
-    if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(chol_inv_kernel), dim3(grid), dim3(kCholThreads),
-                                    args, kCholSmem, st) != cudaSuccess)
-      return GPTQ_ERR_CUDA;
-    count_launch();
-    return GPTQ_OK;
-  };
-  float* Ahi = reinterpret_cast<float*>(w + l.ahi);
-  float* Alo = reinterpret_cast<float*>(w + l.alo);
-  float* Bhi = reinterpret_cast<float*>(w + l.bhi);
-  float* Blo = reinterpret_cast<float*>(w + l.blo);
-  float* P = reinterpret_cast<float*>(w + l.panel);
-  const int nb_outer = n >= kBlockedMinN ? kNB : n;  // one block: the cooperative kernel alone
-  for (int k0 = 0; k0 < n; k0 += nb_outer) {
-    const int kb = std::min(nb_outer, n - k0), k1 = k0 + kb, m = n - k1;
-    const int kp = static_cast<int>(ceil_div(kb, 32)) * 32;  // padded contraction length
-    float* XK = U + static_cast<int64_t>(k0) * n;             // block row K of X (and of R)
-    float* XKK = XK + k0;
-    gptq_status s = factor_block(k0, kb);
-    if (s != GPTQ_OK) return s;
-    if (k0 > 0) {
-      // finalize: X_K,<K = X_KK R_K,<K  (R_K,<K split, then its place zeroed)
-      if ((s = split_cols_tf32(XK, n, kb, k0, kp, 1.0f, Bhi, Blo, st)) != GPTQ_OK) return s;
-      if (cudaMemset2DAsync(XK, static_cast<size_t>(n) * 4, 0, static_cast<size_t>(k0) * 4, kb, st) != cudaSuccess)
-        return GPTQ_ERR_CUDA;
-      if ((s = split_rows_tf32(XKK, n, kb, kb, kp, -1.0f, Ahi, Alo, st)) != GPTQ_OK) return s;
-      if ((s = gemm_nt_tc(XK, n, kb, k0, kp, Ahi, Alo, Bhi, Blo, st)) != GPTQ_OK) return s;
-    }
-    if (m == 0) break;
-    // panel: L_>K,K = A_>K,K X_KK^T into P [m, kp]
-    float* AIK = A + static_cast<int64_t>(k1) * n + k0;
-    if ((s = split_rows_tf32(AIK, n, m, kb, kp, -1.0f, Ahi, Alo, st)) != GPTQ_OK) return s;
-    if ((s = split_rows_tf32(XKK, n, kb, kb, kp, 1.0f, Bhi, Blo, st)) != GPTQ_OK) return s;
-    if (cudaMemsetAsync(P, 0, static_cast<size_t>(m) * kp * sizeof(float), st) != cudaSuccess) return GPTQ_ERR_CUDA;
-    if ((s = gemm_nt_tc(P, kp, m, kb, kp, Ahi, Alo, Bhi, Blo, st)) != GPTQ_OK) return s;
-    // trailing update: A_>K,>K -= P P^T
-    if ((s = split_rows_tf32(P, kp, m, kb, kp, 1.0f, Ahi, Alo, st)) != GPTQ_OK) return s;
-    if ((s = gemm_nt_tc(A + static_cast<int64_t>(k1) * n + k1, n, m, m, kp, Ahi, Alo, Ahi, Alo, st)) != GPTQ_OK)
-      return s;
-    // inverse update: R_>K,<=K -= P X_K,<=K
-    if ((s = split_cols_tf32(XK, n, kb, k1, kp, 1.0f, Bhi, Blo, st)) != GPTQ_OK) return s;
-    if ((s = gemm_nt_tc(U + static_cast<int64_t>(k1) * n, n, m, k1, kp, Ahi, Alo, Bhi, Blo, st)) != GPTQ_OK)
-      return s;
-  }
-  {
-    const int64_t count = static_cast<int64_t>(n) * n;
-    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(ceil_div(count / 2, 256), 148 * 16));
-    launch(reverse_kernel, static_cast<unsigned>(blocks), 256, 0, st, U, count);
-    if (launch_status() != GPTQ_OK) return GPTQ_ERR_CUDA;
-  }
+  CholArgs ca;
+  ca.A = A;
+  ca.Y = Y;
+  ca.Linv = reinterpret_cast<float*>(w + l.linv);
+  ca.ld = np;
+  ca.nb = static_cast<int>(np / kT);
+  ca.fstatus = fstatus;
+  ca.bar = bar;
+  ca.abort = reinterpret_cast<int*>(bar + 2);
+  ca.wait_ns = wait_limit_ns();
+  void* args[] = {&ca};
+  if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(chol_tc_kernel), dim3(grid), dim3(kCholThreads), args,
+                                  kCholSmem, st) != cudaSuccess)
+    return GPTQ_ERR_CUDA;
+  count_launch();
+  launch(anti_transpose_kernel, dim3(static_cast<unsigned>(ceil_div(n, 32)), static_cast<unsigned>(ceil_div(n, 32))),
+         dim3(32, 8), 0, st, Y, np, n, U);
+  if (launch_status() != GPTQ_OK) return GPTQ_ERR_CUDA;
 
   int fs = 0;
   if (cudaMemcpyAsync(&fs, fstatus, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return GPTQ_ERR_CUDA;

@@ -45,15 +45,6 @@ constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 constexpr size_t kSmemBytes = 1024 + size_t(kStages) * kStageBytes + 256;
 constexpr uint64_t kDrainNs = 2000000000ull;
-// K chunks (of kBK) per accumulation unit in the factorization's GEMMs: each
-// unit's product goes through tensor memory on its own and is subtracted from
-// the output in fp32 by the epilogue (one read-modify-write of the tile per
-// unit, L2-resident for consecutive units of a tile).  The tensor-core
-// accumulator rounds like truncation, so its error grows with the number of
-// MMAs it sums; 128 columns of K keep it near an fp32 product's.  The column
-// loop's updates use one unit for the whole K (<= 1024), which its parity
-// tests show to be accurate enough, and save the extra passes over W.
-constexpr int kGemmUnitChunks = 4;
 
 struct TrailParams {
   float* W;        // [M, ldw]
@@ -297,43 +288,6 @@ __global__ void split_transpose_tf32_kernel(const float* __restrict__ U, int n, 
   }
 }
 
-// hi[i][k] / lo[i][k] (i < rows, k < kpad, pitch kpad) = tf32 split of
-// sign * src[i][k] for k < cols, zero for cols <= k < kpad.
-__global__ void split_rows_tf32_kernel(const float* __restrict__ src, int64_t lds, int rows, int cols, int kpad,
-                                       float sign, float* __restrict__ hi, float* __restrict__ lo) {
-  const int i = blockIdx.y;
-  if (i >= rows) return;
-  for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < kpad; k += gridDim.x * blockDim.x) {
-    const float x = k < cols ? sign * src[static_cast<int64_t>(i) * lds + k] : 0.0f;
-    const float h = __uint_as_float(__float_as_uint(x) & 0xffffe000u);
-    hi[static_cast<int64_t>(i) * kpad + k] = h;
-    lo[static_cast<int64_t>(i) * kpad + k] = x - h;
-  }
-}
-
-// hi[j][k] / lo[j][k] (j < cols, k < kpad, pitch kpad) = tf32 split of
-// sign * src[k][j] for k < rows, zero beyond: the transpose, through 32 x 32
-// shared-memory tiles.
-__global__ void split_cols_tf32_kernel(const float* __restrict__ src, int64_t lds, int rows, int cols, int kpad,
-                                       float sign, float* __restrict__ hi, float* __restrict__ lo) {
-  __shared__ float t[32][33];
-  const int k0 = blockIdx.y * 32, j0 = blockIdx.x * 32;
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    const int k = k0 + i, j = j0 + threadIdx.x;
-    t[i][threadIdx.x] = (k < rows && j < cols) ? sign * src[static_cast<int64_t>(k) * lds + j] : 0.0f;
-  }
-  __syncthreads();
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    const int j = j0 + i, k = k0 + threadIdx.x;
-    if (j < cols && k < kpad) {
-      const float x = t[threadIdx.x][i];
-      const float h = __uint_as_float(__float_as_uint(x) & 0xffffe000u);
-      hi[static_cast<int64_t>(j) * kpad + k] = h;
-      lo[static_cast<int64_t>(j) * kpad + k] = x - h;
-    }
-  }
-}
-
 bool set_smem_attr(const DeviceInfo* info) {
   static std::atomic<bool> attr_set[64] = {};  // per device, shared by host threads
   if (!attr_set[info->device]) {
@@ -395,61 +349,5 @@ gptq_status trailing_update_tc(float* W, int64_t ldw, int M, int N, int K, int c
   return launch_status();
 }
 
-
-gptq_status split_rows_tf32(const float* src, int64_t lds, int rows, int cols, int kpad, float sign, float* hi,
-                            float* lo, cudaStream_t st) {
-  if (rows <= 0 || kpad <= 0) return GPTQ_OK;
-  const dim3 grid(static_cast<unsigned>(std::min<int64_t>(ceil_div(kpad, 256), 8)), static_cast<unsigned>(rows));
-  launch(split_rows_tf32_kernel, grid, 256, 0, st, src, lds, rows, cols, kpad, sign, hi, lo);
-  return launch_status();
-}
-
-gptq_status split_cols_tf32(const float* src, int64_t lds, int rows, int cols, int kpad, float sign, float* hi,
-                            float* lo, cudaStream_t st) {
-  if (cols <= 0 || kpad <= 0) return GPTQ_OK;
-  const dim3 grid(static_cast<unsigned>(ceil_div(cols, 32)), static_cast<unsigned>(ceil_div(kpad, 32)));
-  launch(split_cols_tf32_kernel, grid, dim3(32, 8), 0, st, src, lds, rows, cols, kpad, sign, hi, lo);
-  return launch_status();
-}
-
-// C[M, N] -= A[M, K] B[N, K]^T (fp32-accurate), A and B given as tf32 hi / lo
-// halves, row-major with K contiguous and row pitch kpad (a multiple of 32,
-// zero-padded past K).  C has row pitch ldc; any alignment.
-gptq_status gemm_nt_tc(float* C, int64_t ldc, int M, int N, int kpad, const float* A_hi, const float* A_lo,
-                       const float* B_hi, const float* B_lo, cudaStream_t st) {
-  const DeviceInfo* info = device_info();
-  if (info == nullptr) return GPTQ_ERR_CUDA;
-  if (M <= 0 || N <= 0 || kpad <= 0) return GPTQ_OK;
-  if (kpad % kBK != 0) return GPTQ_ERR_INVALID_ARG;
-  if (!set_smem_attr(info)) return GPTQ_ERR_CUDA;
-  const CUtensorMapDataType f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-  const uint64_t pitch = static_cast<uint64_t>(kpad) * 4;
-  CUtensorMap m_ahi, m_alo, m_bhi, m_blo;
-  if (!make_tensor_map_2d(&m_ahi, f32, A_hi, kpad, static_cast<uint64_t>(M), pitch, kBK, kBM,
-                          CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tensor_map_2d(&m_alo, f32, A_lo, kpad, static_cast<uint64_t>(M), pitch, kBK, kBM,
-                          CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tensor_map_2d(&m_bhi, f32, B_hi, kpad, static_cast<uint64_t>(N), pitch, kBK, kBN,
-                          CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tensor_map_2d(&m_blo, f32, B_lo, kpad, static_cast<uint64_t>(N), pitch, kBK, kBN,
-                          CU_TENSOR_MAP_SWIZZLE_128B))
-    return GPTQ_ERR_CUDA;
-  TrailParams p;
-  p.W = C;
-  p.ldw = ldc;
-  p.M = M;
-  p.N = N;
-  p.K = kpad;
-  p.unit_chunks = kGemmUnitChunks;
-  p.c0 = 0;
-  p.k0 = 0;
-  p.tiles_m = static_cast<int>(ceil_div(M, kBM));
-  p.tiles_n = static_cast<int>(ceil_div(N, kBN));
-  p.status = info->status;
-  p.wait_ns = wait_limit_ns();
-  const int grid = std::min(info->sm_count, p.tiles_m * p.tiles_n);
-  launch(trailing_tc_kernel, grid, kThreads, kSmemBytes, st, m_ahi, m_alo, m_bhi, m_blo, p);
-  return launch_status();
-}
 
 }  // namespace gptq
