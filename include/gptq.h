@@ -91,6 +91,27 @@ uint64_t gptq_kernel_launches(void);
  * first failure since the last read is kept. */
 gptq_status gptq_get_device_status(void* stream);
 
+/* Tracing: per-kernel device time.
+ *
+ * The pages have no counterpart to this; it is the measurement hook that
+ * reports where a layer pass spends its time.  While enabled, every kernel
+ * this library launches (from any host thread) is bracketed by two CUDA
+ * events recorded on its stream; the events cost a few microseconds of host
+ * time per launch, so leave tracing off in timed work.
+ * gptq_trace_read waits for the recorded launches to finish and writes, per
+ * kernel (name without namespaces and parameters, e.g.
+ * "gptq_block_kernel<16>"), the launches and the summed device milliseconds
+ * since the previous read into out[0 .. max_entries), largest time first.  It
+ * returns the number of entries written (at most max_entries), or -1 if an
+ * event could not be read (the records are dropped either way). */
+typedef struct {
+  char name[64];
+  uint64_t launches;
+  double ms;
+} gptq_trace_entry;
+void gptq_trace_enable(int32_t on);
+int32_t gptq_trace_read(gptq_trace_entry* out, int32_t max_entries);
+
 /* Bound, in nanoseconds, on every in-kernel pipeline wait of later launches
  * (default 2 s; UINT64_MAX restores the default).  A wait that runs out
  * records GPTQ_ERR_TIMEOUT in the device status word; the kernel then lets its

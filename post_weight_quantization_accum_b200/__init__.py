@@ -10,7 +10,7 @@ import ctypes
 
 import torch
 
-from ._lib import GPTQ_BF16, GPTQ_F32, LIB, GptqError, check  # noqa: F401
+from ._lib import GPTQ_BF16, GPTQ_F32, LIB, GptqError, TraceEntry, check  # noqa: F401
 
 __all__ = [
     "GptqError",
@@ -26,6 +26,8 @@ __all__ = [
     "gptq_get_device_status",
     "gptq_set_wait_limit_ns",
     "gptq_kernel_launches",
+    "gptq_trace_enable",
+    "gptq_trace_read",
     "workspace",
     "quantize_layer",
     "quantize_layer_group",
@@ -69,6 +71,20 @@ def gptq_set_wait_limit_ns(ns):
 
 def gptq_kernel_launches():
     return int(LIB.gptq_kernel_launches())
+
+
+def gptq_trace_enable(on=True):
+    LIB.gptq_trace_enable(1 if on else 0)
+
+
+def gptq_trace_read(max_entries=64):
+    """{kernel name: (launches, device ms)} since the previous read (waits for
+    the traced launches to finish)."""
+    buf = (TraceEntry * max_entries)()
+    n = LIB.gptq_trace_read(buf, max_entries)
+    if n < 0:
+        raise GptqError("gptq_trace_read", 4)
+    return {buf[i].name.decode(): (int(buf[i].launches), float(buf[i].ms)) for i in range(n)}
 
 
 def gptq_hessian_accum(H, X, alpha, hdiag=None, ws=None, stream=None):

@@ -31,6 +31,8 @@ _SIGS = {
     "gptq_kernel_launches": (ctypes.c_uint64, []),
     "gptq_get_device_status": (ctypes.c_int, [_P]),
     "gptq_set_wait_limit_ns": (None, [ctypes.c_uint64]),
+    "gptq_trace_enable": (None, [ctypes.c_int32]),
+    "gptq_trace_read": (ctypes.c_int32, [_P, ctypes.c_int32]),
     "gptq_hessian_workspace_size": (ctypes.c_size_t, [ctypes.c_int32, ctypes.c_int64]),
     "gptq_hessian_accum": (ctypes.c_int, [_P, _P, _P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int64,
                                           ctypes.c_float, _P, ctypes.c_size_t, _P]),
@@ -55,6 +57,11 @@ _SIGS = {
                                     ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _P, _P, _P, ctypes.c_size_t,
                                     _P]),
 }
+
+
+class TraceEntry(ctypes.Structure):
+    """gptq_trace_entry: one kernel's launches and summed device milliseconds."""
+    _fields_ = [("name", ctypes.c_char * 64), ("launches", ctypes.c_uint64), ("ms", ctypes.c_double)]
 
 
 class GptqError(RuntimeError):

@@ -1,10 +1,16 @@
 // C ABI of the library: argument validation, per-device state and dispatch to
 // the kernels in hessian.cu, hinv.cu, quantize.cu, pack.cu, matvec.cu and round2d.cu.  Nothing here
 // allocates device memory; every scratch byte comes from the caller.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstring>
+#include <cstdlib>
+#include <cxxabi.h>
+#include <map>
 #include <mutex>
+#include <string>
+#include <vector>
 
 #include "common.cuh"
 
@@ -105,6 +111,92 @@ uint64_t wait_limit_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
 static std::atomic<uint64_t> g_launches{0};
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
+// ---------------------------------------------------------------------------
+// tracing: per-kernel device time from CUDA events around each launch
+// ---------------------------------------------------------------------------
+
+namespace {
+
+struct TraceRec {
+  cudaEvent_t begin, end;
+  const void* kernel;
+  int device;
+};
+
+std::atomic<bool> g_trace{false};
+std::mutex g_trace_mutex;
+std::vector<TraceRec> g_trace_recs;                          // launches not yet read
+std::vector<std::pair<int, cudaEvent_t>> g_trace_free;       // (device, event) ready for reuse
+thread_local cudaEvent_t t_trace_begin = nullptr;            // this thread's launch in progress
+
+cudaEvent_t trace_event(int dev) {  // caller holds g_trace_mutex
+  for (size_t i = 0; i < g_trace_free.size(); ++i)
+    if (g_trace_free[i].first == dev) {
+      cudaEvent_t e = g_trace_free[i].second;
+      g_trace_free[i] = g_trace_free.back();
+      g_trace_free.pop_back();
+      return e;
+    }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+// "gptq::(anonymous namespace)::gptq_block_kernel<16>(gptq::...)" -> "gptq_block_kernel<16>"
+std::string short_kernel_name(const void* kernel) {
+  const char* mangled = nullptr;
+  if (cudaFuncGetName(&mangled, kernel) != cudaSuccess || mangled == nullptr) return "unknown";
+  int ok = -1;
+  char* dem = abi::__cxa_demangle(mangled, nullptr, nullptr, &ok);
+  std::string name = (ok == 0 && dem != nullptr) ? dem : mangled;
+  std::free(dem);
+  int depth = 0;  // drop the parameter list: the first '(' outside template brackets
+  for (size_t i = 0; i < name.size(); ++i) {
+    if (name[i] == '<') ++depth;
+    if (name[i] == '>') --depth;
+    if (name[i] == '(' && depth == 0 && i > 0 && name.compare(i, 20, "(anonymous namespace") != 0) {
+      name.resize(i);
+      break;
+    }
+  }
+  const std::string ns[] = {"gptq::(anonymous namespace)::", "gptq::"};
+  for (const std::string& p : ns)
+    for (size_t at; (at = name.find(p)) != std::string::npos;) name.erase(at, p.size());
+  return name;
+}
+
+}  // namespace
+
+bool trace_on() { return g_trace.load(std::memory_order_relaxed); }
+
+void trace_begin(cudaStream_t st) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return;
+  std::lock_guard<std::mutex> lock(g_trace_mutex);
+  cudaEvent_t e = trace_event(dev);
+  if (e != nullptr && cudaEventRecord(e, st) != cudaSuccess) {
+    g_trace_free.emplace_back(dev, e);
+    e = nullptr;
+  }
+  t_trace_begin = e;
+}
+
+void trace_end(cudaStream_t st, const void* kernel) {
+  cudaEvent_t b = t_trace_begin;
+  t_trace_begin = nullptr;
+  if (b == nullptr) return;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return;
+  std::lock_guard<std::mutex> lock(g_trace_mutex);
+  cudaEvent_t e = trace_event(dev);
+  if (e == nullptr || cudaEventRecord(e, st) != cudaSuccess) {
+    g_trace_free.emplace_back(dev, b);
+    if (e != nullptr) g_trace_free.emplace_back(dev, e);
+    return;
+  }
+  g_trace_recs.push_back({b, e, kernel, dev});
+}
+
 }  // namespace gptq
 
 using namespace gptq;
@@ -137,6 +229,41 @@ uint64_t gptq_kernel_launches(void) { return g_launches.load(std::memory_order_r
 
 void gptq_set_wait_limit_ns(uint64_t ns) {
   g_wait_ns.store(ns == UINT64_MAX ? kDefaultWaitNs : ns, std::memory_order_relaxed);
+}
+
+void gptq_trace_enable(int32_t on) { g_trace.store(on != 0, std::memory_order_relaxed); }
+
+int32_t gptq_trace_read(gptq_trace_entry* out, int32_t max_entries) {
+  std::lock_guard<std::mutex> lock(g_trace_mutex);
+  std::map<const void*, std::pair<uint64_t, double>> sums;
+  int err = 0;
+  for (const TraceRec& r : g_trace_recs) {
+    float ms = 0.0f;
+    if (cudaEventSynchronize(r.end) != cudaSuccess || cudaEventElapsedTime(&ms, r.begin, r.end) != cudaSuccess)
+      err = 1;
+    auto& acc = sums[r.kernel];
+    acc.first += 1;
+    acc.second += ms;
+    g_trace_free.emplace_back(r.device, r.begin);
+    g_trace_free.emplace_back(r.device, r.end);
+  }
+  g_trace_recs.clear();
+  if (err) return -1;
+  std::vector<gptq_trace_entry> entries;
+  for (const auto& kv : sums) {
+    gptq_trace_entry e{};
+    const std::string name = short_kernel_name(kv.first);
+    std::strncpy(e.name, name.c_str(), sizeof(e.name) - 1);
+    e.launches = kv.second.first;
+    e.ms = kv.second.second;
+    entries.push_back(e);
+  }
+  std::sort(entries.begin(), entries.end(), [](const gptq_trace_entry& a, const gptq_trace_entry& b) {
+    return a.ms > b.ms;
+  });
+  const int32_t n = static_cast<int32_t>(std::min<size_t>(entries.size(), max_entries > 0 ? max_entries : 0));
+  for (int32_t i = 0; i < n; ++i) out[i] = entries[i];
+  return n;
 }
 
 gptq_status gptq_get_device_status(void* stream) {

@@ -281,6 +281,12 @@ __host__ __device__ constexpr uint32_t instr_desc(uint32_t fmt, uint32_t a_mn_ma
          ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
+// dst[0..3] += v as one L2 vector reduction (dst 16-byte aligned).
+__device__ __forceinline__ void red_add_v4(float* dst, float4 v) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+               : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // host helpers
 // ---------------------------------------------------------------------------
@@ -309,10 +315,19 @@ inline gptq_status launch_status() {
 // Number of kernels this library has launched in the process.
 void count_launch();
 
-// Launches `kernel` and counts it.
+// Tracing (gptq_trace_enable): while it is on, every launch is bracketed by
+// two CUDA events on its stream, trace_begin before and trace_end after.
+bool trace_on();
+void trace_begin(cudaStream_t st);
+void trace_end(cudaStream_t st, const void* kernel);
+
+// Launches `kernel` and counts it (and traces it when tracing is on).
 template <typename... KArgs, typename... Args>
 inline void launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+  const bool traced = trace_on();
+  if (traced) trace_begin(st);
   kernel<<<grid, block, smem, st>>>(static_cast<KArgs>(args)...);
+  if (traced) trace_end(st, reinterpret_cast<const void*>(kernel));
   count_launch();
 }
 

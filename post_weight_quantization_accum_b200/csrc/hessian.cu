@@ -423,7 +423,10 @@ gptq_status hessian_accum(float* H, double* hdiag, const void* X, int64_t n_tok,
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  const bool traced = trace_on();
+  if (traced) trace_begin(stream);
   if (cudaLaunchKernelEx(&cfg, syrk_tc_kernel, xmap, p) != cudaSuccess) return GPTQ_ERR_CUDA;
+  if (traced) trace_end(stream, reinterpret_cast<const void*>(syrk_tc_kernel));
   count_launch();
   launch(syrk_finalize_kernel, dim3(p.tiles, kTile / 32, kTile / 32), dim3(32, 8), 0, stream, partial, H, n, p.tiles,
                                                                                         p.splits, alpha);

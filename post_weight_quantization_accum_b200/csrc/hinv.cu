@@ -342,11 +342,6 @@ __device__ __forceinline__ void issue_chunk(const uint8_t* stage, uint32_t d_tme
   }
 }
 
-__device__ __forceinline__ void red4(float* dst, float4 v) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
-               : "memory");
-}
-
 // The accumulator into the output tile: warp w reads lanes 32 (w % 4) .. + 31
 // (tile rows) and columns 64 (w / 4) .. + 63, and stores them (or subtracts
 // them as L2 reductions, so the old values never travel to the SM).
@@ -365,7 +360,7 @@ __device__ __forceinline__ void write_tile(const TileOp& op, int64_t ld, uint32_
       const float4 f = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
                                    __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
       if (op.sub)
-        red4(row + c0 + 4 * q, make_float4(-f.x, -f.y, -f.z, -f.w));
+        red_add_v4(row + c0 + 4 * q, make_float4(-f.x, -f.y, -f.z, -f.w));
       else
         *reinterpret_cast<float4*>(row + c0 + 4 * q) = f;
     }
@@ -834,9 +829,12 @@ gptq_status prepare_hinv(const float* H, const double* hdiag, int n, float damp,
   ca.abort = reinterpret_cast<int*>(bar + 2);
   ca.wait_ns = wait_limit_ns();
   void* args[] = {&ca};
+  const bool traced = trace_on();
+  if (traced) trace_begin(st);
   if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(chol_tc_kernel), dim3(grid), dim3(kCholThreads), args,
                                   kCholSmem, st) != cudaSuccess)
     return GPTQ_ERR_CUDA;
+  if (traced) trace_end(st, reinterpret_cast<const void*>(chol_tc_kernel));
   count_launch();
   launch(anti_transpose_kernel, dim3(static_cast<unsigned>(ceil_div(n, 32)), static_cast<unsigned>(ceil_div(n, 32))),
          dim3(32, 8), 0, st, Y, np, n, U);

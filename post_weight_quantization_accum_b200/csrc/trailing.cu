@@ -231,23 +231,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(buf * kBN + c), v);
         tmem_ld_wait();
         if (row < p.M && c < ncols) {
+          // W -= acc as L2 reductions: nothing is read back into the SM, so
+          // the epilogue does not wait on L2 latency; each element receives
+          // one fp32 addition per launch (tiles are disjoint), the result of
+          // a load, an fp32 subtraction and a store
           if (vec && c + 32 <= ncols) {
-            float4* w4 = reinterpret_cast<float4*>(wrow + c);
-            float4 cur[8];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) cur[q] = w4[q];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              cur[q].x -= __uint_as_float(v[4 * q]);
-              cur[q].y -= __uint_as_float(v[4 * q + 1]);
-              cur[q].z -= __uint_as_float(v[4 * q + 2]);
-              cur[q].w -= __uint_as_float(v[4 * q + 3]);
-              w4[q] = cur[q];
-            }
+            for (int q = 0; q < 8; ++q)
+              red_add_v4(wrow + c + 4 * q, make_float4(-__uint_as_float(v[4 * q]), -__uint_as_float(v[4 * q + 1]),
+                                                       -__uint_as_float(v[4 * q + 2]), -__uint_as_float(v[4 * q + 3])));
           } else {
 #pragma unroll
             for (int q = 0; q < 32; ++q)
-              if (c + q < ncols) wrow[c + q] -= __uint_as_float(v[q]);
+              if (c + q < ncols) atomicAdd(wrow + c + q, -__uint_as_float(v[q]));
           }
         }
       }
