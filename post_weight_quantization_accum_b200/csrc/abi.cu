@@ -159,6 +159,7 @@ std::string short_kernel_name(const void* kernel) {
       break;
     }
   }
+  if (name.compare(0, 5, "void ") == 0) name.erase(0, 5);  // template instances carry their return type
   const std::string ns[] = {"gptq::(anonymous namespace)::", "gptq::"};
   for (const std::string& p : ns)
     for (size_t at; (at = name.find(p)) != std::string::npos;) name.erase(at, p.size());

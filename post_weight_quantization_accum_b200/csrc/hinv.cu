@@ -181,7 +181,7 @@ constexpr uint64_t kDrainNs = 2000000000ull;
 struct CholArgs {
   float* A;         // [np, np] at pitch ld, lower: the damped reversed matrix; panels become L
   float* Y;         // [np, np] at pitch ld, zero on entry: becomes Y = (L^-1)^T (upper)
-  float* Linv;      // [kT, kT] the current diagonal block's inverse, row-major
+  float* Linv;      // [2][kT, kT] diagonal block k's inverse (row-major) in slot k % 2
   int64_t ld;       // np, a multiple of kT
   int nb;           // np / kT
   int* fstatus;     // factorization status word
@@ -190,12 +190,15 @@ struct CholArgs {
   uint64_t wait_ns;
 };
 
-// Time-bounded barrier over the whole (co-resident) grid.
-__device__ bool grid_sync(const CholArgs& p) {
-  __shared__ int ok_s;
+// Grid barrier over the whole (co-resident) grid in two halves: grid_arrive
+// (every thread of the CTA; its writes so far become visible first) returns
+// the generation that grid_wait then waits to see pass (time-bounded).  A CTA
+// may work between the two.
+__device__ unsigned grid_arrive(const CholArgs& p) {
+  __shared__ unsigned gen_s;
+  __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
-    int ok = 1;
     volatile unsigned* gen_p = p.bar + 1;
     const unsigned gen = *gen_p;
     __threadfence();
@@ -203,19 +206,29 @@ __device__ bool grid_sync(const CholArgs& p) {
       atomicExch(p.bar, 0u);
       __threadfence();
       atomicAdd(p.bar + 1, 1u);
-    } else {
-      const uint64_t t0 = global_ns();
-      while (*gen_p == gen) {
-        if (*reinterpret_cast<volatile int*>(p.abort)) {
-          ok = 0;
-          break;
-        }
-        if (global_ns() - t0 > p.wait_ns) {
-          set_status(p.fstatus, GPTQ_ERR_TIMEOUT);
-          atomicExch(p.abort, 1);
-          ok = 0;
-          break;
-        }
+    }
+    gen_s = gen;
+  }
+  __syncthreads();
+  return gen_s;
+}
+
+__device__ bool grid_wait(const CholArgs& p, unsigned gen) {
+  __shared__ int ok_s;
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    volatile unsigned* gen_p = p.bar + 1;
+    const uint64_t t0 = global_ns();
+    while (*gen_p == gen) {
+      if (*reinterpret_cast<volatile int*>(p.abort)) {
+        ok = 0;
+        break;
+      }
+      if (global_ns() - t0 > p.wait_ns) {
+        set_status(p.fstatus, GPTQ_ERR_TIMEOUT);
+        atomicExch(p.abort, 1);
+        ok = 0;
+        break;
       }
     }
     __threadfence();
@@ -224,6 +237,8 @@ __device__ bool grid_sync(const CholArgs& p) {
   __syncthreads();
   return ok_s != 0;
 }
+
+__device__ __forceinline__ bool grid_sync(const CholArgs& p) { return grid_wait(p, grid_arrive(p)); }
 
 __device__ __forceinline__ void give_up(const CholArgs& p) {
   if (threadIdx.x == 0) {
@@ -246,10 +261,12 @@ struct TileOp {
   int sub;
 };
 
+__device__ __forceinline__ float* linv_slot(const CholArgs& p, int k) { return p.Linv + (k & 1) * kT * kT; }
+
 __device__ TileOp op_phase_t(const CholArgs& p, int k, int t) {
   const int ntrsm = p.nb - 1 - k;
   TileOp op;
-  op.Q = p.Linv;
+  op.Q = linv_slot(p, k);
   op.ldq = kT;
   op.ldp = p.ld;
   op.sub = 0;
@@ -479,8 +496,8 @@ __device__ __forceinline__ void solve16(float (&x)[16], const float* S, const fl
   }
 }
 
-// Factors the diagonal block k (by one CTA): Linv_kk into p.Linv (row-major)
-// and Y_kk = Linv_kk^T into Y's diagonal tile.
+// Factors the diagonal block k (by one CTA): Linv_kk into its Linv slot
+// (row-major) and Y_kk = Linv_kk^T into Y's diagonal tile.
 //
 // In 16-wide sub-panels s of the block S (its lower half), with R = I beside it:
 //   warp 0   Cholesky of the sub-panel's 16 x 16 diagonal block (chol16)
@@ -500,11 +517,21 @@ __device__ void factor_block(const CholArgs& p, int k, float* fs) {
   float* rd = Pn + kSub * kT;   // [kT]: 1 / L_jj
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const float* Akk = tile_at(p.A, p.ld, k, k);
-  for (int e = t; e < kT * (kT / 4); e += kCholThreads) {
-    const int r = e >> 5, c = 4 * (e & 31);
-    *reinterpret_cast<float4*>(S + r * kSP + c) = __ldcg(reinterpret_cast<const float4*>(Akk + r * p.ld + c));
-    *reinterpret_cast<float4*>(XR + r * kSP + c) =
-        make_float4(r == c ? 1.0f : 0.0f, r == c + 1 ? 1.0f : 0.0f, r == c + 2 ? 1.0f : 0.0f, r == c + 3 ? 1.0f : 0.0f);
+  {
+    constexpr int kPer = kT * (kT / 4) / kCholThreads;  // float4 per thread
+    float4 a[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {  // every load in flight before the first store
+      const int e = t + u * kCholThreads, r = e >> 5, c = 4 * (e & 31);
+      a[u] = __ldcg(reinterpret_cast<const float4*>(Akk + r * p.ld + c));
+    }
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int e = t + u * kCholThreads, r = e >> 5, c = 4 * (e & 31);
+      *reinterpret_cast<float4*>(S + r * kSP + c) = a[u];
+      *reinterpret_cast<float4*>(XR + r * kSP + c) = make_float4(r == c ? 1.0f : 0.0f, r == c + 1 ? 1.0f : 0.0f,
+                                                                 r == c + 2 ? 1.0f : 0.0f, r == c + 3 ? 1.0f : 0.0f);
+    }
   }
   __syncthreads();
   bool nonfinite = false, notpd = false;
@@ -632,17 +659,26 @@ __device__ void factor_block(const CholArgs& p, int k, float* fs) {
     notpd = __any_sync(0xffffffffu, notpd);
     if (lane == 0 && (nonfinite || notpd)) set_status(p.fstatus, nonfinite ? GPTQ_ERR_NONFINITE : GPTQ_ERR_NOT_PD);
   }
-  // Linv (row-major, zeros above the diagonal) and Y_kk = Linv^T
+  // Linv (row-major, zeros above the diagonal); its transpose staged in S's
+  // place (conflict-free: consecutive threads take consecutive rows of X)
+  for (int e = t; e < kT * (kT / 4); e += kCholThreads) {
+    const int r = e >> 5, c = 4 * (e & 31);
+    float4 x = *reinterpret_cast<const float4*>(XR + r * kSP + c);
+    x = make_float4(c <= r ? x.x : 0.0f, c + 1 <= r ? x.y : 0.0f, c + 2 <= r ? x.z : 0.0f, c + 3 <= r ? x.w : 0.0f);
+    *reinterpret_cast<float4*>(linv_slot(p, k) + r * kT + c) = x;
+    const int rt = e & (kT - 1), ct = 4 * (e >> 7);
+    const float4 xt = *reinterpret_cast<const float4*>(XR + rt * kSP + ct);
+    S[ct * kSP + rt] = ct <= rt ? xt.x : 0.0f;
+    S[(ct + 1) * kSP + rt] = ct + 1 <= rt ? xt.y : 0.0f;
+    S[(ct + 2) * kSP + rt] = ct + 2 <= rt ? xt.z : 0.0f;
+    S[(ct + 3) * kSP + rt] = ct + 3 <= rt ? xt.w : 0.0f;
+  }
+  __syncthreads();
+  // Y_kk = Linv^T, row by row
   float* Ykk = tile_at(p.Y, p.ld, k, k);
   for (int e = t; e < kT * (kT / 4); e += kCholThreads) {
     const int r = e >> 5, c = 4 * (e & 31);
-    const float4 x = *reinterpret_cast<const float4*>(XR + r * kSP + c);
-    *reinterpret_cast<float4*>(p.Linv + r * kT + c) =
-        make_float4(c <= r ? x.x : 0.0f, c + 1 <= r ? x.y : 0.0f, c + 2 <= r ? x.z : 0.0f, c + 3 <= r ? x.w : 0.0f);
-    const int ry = e & (kT - 1), cy = 4 * (e >> 7);  // Y_kk[ry][cy + u] = X[cy + u][ry]
-    *reinterpret_cast<float4*>(Ykk + ry * p.ld + cy) =
-        make_float4(cy >= ry ? XR[cy * kSP + ry] : 0.0f, cy + 1 >= ry ? XR[(cy + 1) * kSP + ry] : 0.0f,
-                    cy + 2 >= ry ? XR[(cy + 2) * kSP + ry] : 0.0f, cy + 3 >= ry ? XR[(cy + 3) * kSP + ry] : 0.0f);
+    *reinterpret_cast<float4*>(Ykk + r * p.ld + c) = *reinterpret_cast<const float4*>(S + r * kSP + c);
   }
   __threadfence();
   __syncthreads();
@@ -686,33 +722,46 @@ __global__ void __launch_bounds__(kCholThreads, 1) chol_tc_kernel(CholArgs p) {
   if (b == 0) factor_block(p, 0, fs);
   bool live = grid_sync(p);
   for (int k = 0; k < nb && live; ++k) {
-    {  // phase T(k)
+    const int m = nb - 1 - k;
+    // Phase T(k).  CTA 0 takes the trsm of row block k+1 (operation 0), then
+    // arrives, then, while the others finish the panel, updates tile
+    // (k+1, k+1) with it (operation 0 of phase U) and factors block k+1 (its
+    // inverse goes to the other Linv slot): the diagonal chain overlaps the
+    // panel's products.
+    if (G == 1) {
+      live = run_ops<false>(p, pp, k, 0, nb - 1);
+    } else if (b == 0) {
+      live = run_ops<false>(p, pp, k, 0, m > 0 ? 1 : 0);
+    } else {
       int lo, hi;
-      share(nb - 1, b, G, lo, hi);
-      live = run_ops<false>(p, pp, k, lo, hi);
-      __threadfence();
-      if (live) live = grid_sync(p);
+      share(nb - 1 - (m > 0 ? 1 : 0), b - 1, G - 1, lo, hi);
+      const int off = m > 0 ? 1 : 0;
+      live = run_ops<false>(p, pp, k, off + lo, off + hi);
     }
     if (!live) break;
-    {  // phase U(k): CTA 0 updates tile (k+1, k+1) and factors it while the others share the rest
-      const int m = nb - 1 - k;
-      const int total = m * (m + 1) / 2 + m * (k + 1);
-      if (G == 1) {
-        live = run_ops<true>(p, pp, k, 0, total);
-        if (live && m > 0) factor_block(p, k + 1, fs);
-      } else if (b == 0) {
-        live = run_ops<true>(p, pp, k, 0, total > 0 ? 1 : 0);
-        __threadfence();
-        __syncthreads();
-        if (live && m > 0) factor_block(p, k + 1, fs);
-      } else if (total > 1) {
-        int lo, hi;
-        share(total - 1, b - 1, G - 1, lo, hi);
-        live = run_ops<true>(p, pp, k, 1 + lo, 1 + hi);
-      }
+    unsigned gen = grid_arrive(p);
+    if (G > 1 && b == 0 && m > 0) {
+      live = run_ops<true>(p, pp, k, 0, 1);
       __threadfence();
-      if (live) live = grid_sync(p);
+      __syncthreads();
+      if (live) factor_block(p, k + 1, fs);
     }
+    if (!live || !grid_wait(p, gen)) {
+      live = false;
+      break;
+    }
+    // Phase U(k): every other update and inverse operation, shared by the
+    // CTAs other than CTA 0 (all of them when there is only one CTA).
+    const int total = m * (m + 1) / 2 + m * (k + 1);
+    if (G == 1) {
+      live = run_ops<true>(p, pp, k, 0, total);
+      if (live && m > 0) factor_block(p, k + 1, fs);
+    } else if (b > 0 && total > 1) {
+      int lo, hi;
+      share(total - 1, b - 1, G - 1, lo, hi);
+      live = run_ops<true>(p, pp, k, 1 + lo, 1 + hi);
+    }
+    if (live) live = grid_sync(p);
   }
   // every exit: this CTA's tensor-core work done, then its tensor memory released
   if (threadIdx.x == 0) {
@@ -745,7 +794,7 @@ PrepLayout prep_layout(int n) {
   l.y = off;
   off += align256(nn);
   l.linv = off;
-  off += align256(static_cast<size_t>(kT) * kT * sizeof(float));
+  off += align256(2 * static_cast<size_t>(kT) * kT * sizeof(float));
   l.key = off;
   off += align256(static_cast<size_t>(n) * sizeof(double));
   l.dead = off;

@@ -31,10 +31,36 @@ def test_reference_arm_prints_one_contract_line():
 def test_stage_rooflines_arithmetic():
     sys.path.insert(0, ROOT)
     import bench
+    pk = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
     r = bench.stage_rooflines({"hessian": 3.0, "prepare_hinv": 2.0, "quantize_layer": 1.0, "pack": 0.01},
-                              rows=4096, n=4096, bits=4, ng=32, sms=148, mhz=2000.0, hbm_gbs=6000.0)
-    assert abs(r["factorization"]["peak"] - 148 * 256 * 2.0e9 / 1e12) < 1e-9
+                              rows=4096, n=4096, bits=4, ng=32, pk=pk)
+    assert r["factorization"]["peak"] == 1600.0
     assert abs(r["factorization"]["achieved"] - 2 * 4096 ** 3 / 3 / 2e-3 / 1e12) < 1e-6
+    assert abs(r["factorization"]["tf32_issue_frac"] - 3 * r["factorization"]["achieved"] / (1600 * 1.1 / 2.25)) < 1e-12
     # codes and zeros read (1 byte each), 512 + 4 packed words per row written
     assert r["pack"]["algorithmic_bytes"] == 4096 * 4096 + 4096 * 32 + 4 * 4096 * (512 + 4)
     assert abs(r["pack"]["frac"] - r["pack"]["achieved"] / 6000.0) < 1e-12
+
+
+def test_trailing_flops_is_the_sum_over_blocks():
+    sys.path.insert(0, ROOT)
+    import bench
+    # square, block-divisible: rows * n * (n - B)
+    assert bench.trailing_flops(4096, 4096, 128) == 4096 * 4096 * (4096 - 128)
+    # ragged: blocks of 128, 128, 44 -> 2 rows (128 * 172 + 128 * 44)
+    assert bench.trailing_flops(10, 300, 128) == 2 * 10 * (128 * 172 + 128 * 44)
+
+
+def test_kernel_rooflines_from_a_trace():
+    sys.path.insert(0, ROOT)
+    import bench
+    pk = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    trace = {"syrk_tc_kernel": (2, 6.0), "chol_tc_kernel": (2, 2.0), "trailing_tc_kernel": (62, 1.0),
+             "gptq_block_kernel<16>": (64, 1.8), "pack_kernel<4>": (4, 0.03)}
+    r = bench.kernel_rooflines(trace, 2, rows=4096, n=4096, n_tok=262144, bits=4, ng=32, block=128, pk=pk,
+                               sms=148, mhz=1965.0)
+    assert r["syrk_tc_kernel"]["ms"] == 3.0 and r["syrk_tc_kernel"]["launches"] == 1
+    assert abs(r["syrk_tc_kernel"]["achieved"] - 4096 * 4097 * 262144 / 3e-3 / 1e12) < 1e-6
+    assert r["gptq_block_kernel"]["launches"] == 32 and abs(r["gptq_block_kernel"]["ms"] - 0.9) < 1e-12
+    assert abs(r["trailing_tc_kernel"]["achieved"] - 4096 * 4096 * 3968 / 0.5e-3 / 1e12) < 1e-6
+    assert r["pack_kernel"]["launches"] == 2
