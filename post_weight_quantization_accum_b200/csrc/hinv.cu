@@ -150,10 +150,11 @@ __global__ void anti_transpose_kernel(const float* __restrict__ Y, int64_t ldy, 
 // (tcgen05.mma kind::tf32, fp32 accumulation in tensor memory), fp32-accurate
 // through the 3-term split P_hi Q_hi + P_hi Q_lo + P_lo Q_hi (x_hi = x with
 // its 13 low mantissa bits cleared, x_lo = x - x_hi; the dropped P_lo Q_lo is
-// below 2^-20 of the product).  Operands are staged through registers (the
-// loads of the next 32-column chunk in flight while the current one is split
-// and stored) into a two-stage shared-memory ring in the 128-byte-swizzled
-// K-major layout; one thread issues the MMAs; the accumulator is
+// below 2^-20 of the product).  The tensor cores read an fp32 operand as tf32
+// by dropping those 13 bits, so the chunks TMA brings in (128-byte swizzle,
+// K-major, a four-stage ring with three chunks in flight ahead) serve as the
+// hi halves as they are, and the threads only form the lo halves (a two-stage
+// ring in the same layout).  One thread issues the MMAs; the accumulator is
 // double-buffered, so one operation's epilogue (tensor memory -> registers ->
 // a store, or an L2 vector reduction for the subtracting operations) overlaps
 // the next one's products.  Each tile receives at most one result per phase.
@@ -165,16 +166,18 @@ constexpr int kT = 128;                      // panel width and tile order
 constexpr int kCk = 32;                      // fp32 columns of K per staged chunk (one 128-byte row)
 constexpr int kChunks = kT / kCk;
 constexpr int kCholThreads = 256;
-constexpr int kBufBytes = kT * kCk * 4;      // one split half of one operand chunk (16 KB)
-constexpr int kStageBytes = 4 * kBufBytes;   // P hi, P lo, Q hi, Q lo
-constexpr int kStages = 2;
+constexpr int kBufBytes = kT * kCk * 4;      // one 128 x 32 fp32 operand chunk (16 KB)
+constexpr int kPairBytes = 2 * kBufBytes;    // a chunk of both operands: P then Q
+constexpr int kRawStages = 4;                // operand chunks as loaded (TMA), 3 in flight ahead
+constexpr int kLoStages = 2;                 // their low halves, formed by the threads
 constexpr int kSP = 132;                     // row pitch (floats) of the diagonal factor's matrices
 constexpr int kSub = 16;                     // sub-panel width of the diagonal factor
-constexpr size_t kRingBytes = static_cast<size_t>(kStages) * kStageBytes;
+constexpr size_t kRingBytes = static_cast<size_t>(kRawStages + kLoStages) * kPairBytes;
 constexpr size_t kFactorBytes = (2 * static_cast<size_t>(kT) * kSP + static_cast<size_t>(kSub) * kT + kT) * 4;
 constexpr size_t kRegionBytes = kFactorBytes > kRingBytes ? kFactorBytes : kRingBytes;
-constexpr size_t kCholSmem = 1024 + kRegionBytes + 128;  // 1024-byte alignment slack, region, barriers
-constexpr uint32_t kCholTmemCols = 2 * kT;               // two 128 x 128 fp32 accumulators
+constexpr int kNumBars = 2 * kRawStages + kLoStages + 2 + 1;  // raw full / free, lo free, accumulators, drain
+constexpr size_t kCholSmem = 1024 + kRegionBytes + kNumBars * 8 + 16;  // alignment slack, region, barriers, slot
+constexpr uint32_t kCholTmemCols = 2 * kT;                         // two 128 x 128 fp32 accumulators
 constexpr int kMaxCholCtas = 1024;
 constexpr uint64_t kDrainNs = 2000000000ull;
 
@@ -252,13 +255,19 @@ __device__ __forceinline__ float* tile_at(float* base, int64_t ld, int i, int j)
 }
 
 // One tile operation: C = P Q^T (sub == 0) or C -= P Q^T (sub == 1); all
-// three are 128 x 128 tiles, rows of P and Q along K.
+// three are 128 x 128 tiles, rows of P and Q along K.  P and Q are given by
+// the tensor map they are loaded through (kMapA, kMapY, kMapL) and the
+// coordinates of their first element.
+enum { kMapA = 0, kMapY = 1, kMapL = 2 };
 struct TileOp {
-  const float* P;
-  const float* Q;
-  int64_t ldp, ldq;
+  int pm, pr, pc;
+  int qm, qr, qc;
   float* C;
   int sub;
+};
+
+struct Maps {
+  const CUtensorMap* m[3];
 };
 
 __device__ __forceinline__ float* linv_slot(const CholArgs& p, int k) { return p.Linv + (k & 1) * kT * kT; }
@@ -266,13 +275,16 @@ __device__ __forceinline__ float* linv_slot(const CholArgs& p, int k) { return p
 __device__ TileOp op_phase_t(const CholArgs& p, int k, int t) {
   const int ntrsm = p.nb - 1 - k;
   TileOp op;
-  op.Q = linv_slot(p, k);
-  op.ldq = kT;
-  op.ldp = p.ld;
+  op.qm = kMapL;
+  op.qr = (k & 1) * kT;  // Linv slot k % 2
+  op.qc = 0;
   op.sub = 0;
-  float* c = t < ntrsm ? tile_at(p.A, p.ld, k + 1 + t, k) : tile_at(p.Y, p.ld, t - ntrsm, k);
-  op.P = c;
-  op.C = c;
+  const bool trsm = t < ntrsm;
+  const int i = trsm ? k + 1 + t : t - ntrsm;
+  op.pm = trsm ? kMapA : kMapY;
+  op.pr = i * kT;
+  op.pc = k * kT;
+  op.C = tile_at(trsm ? p.A : p.Y, p.ld, i, k);
   return op;
 }
 
@@ -280,8 +292,6 @@ __device__ TileOp op_phase_u(const CholArgs& p, int k, int t) {
   const int m = p.nb - 1 - k;
   const int nupd = m * (m + 1) / 2;
   TileOp op;
-  op.ldp = p.ld;
-  op.ldq = p.ld;
   op.sub = 1;
   if (t < nupd) {  // (a, b), b <= a, in row-major order of the lower triangle
     int a = static_cast<int>((sqrtf(8.0f * t + 1.0f) - 1.0f) * 0.5f);
@@ -289,63 +299,40 @@ __device__ TileOp op_phase_u(const CholArgs& p, int k, int t) {
     while (a * (a + 1) / 2 > t) --a;
     const int b = t - a * (a + 1) / 2;
     const int i = k + 1 + a, j = k + 1 + b;
-    op.P = tile_at(p.A, p.ld, i, k);
-    op.Q = tile_at(p.A, p.ld, j, k);
+    op.pm = kMapA, op.pr = i * kT, op.pc = k * kT;  // L_ik
+    op.qm = kMapA, op.qr = j * kT, op.qc = k * kT;  // L_jk
     op.C = tile_at(p.A, p.ld, i, j);
   } else {
     const int tt = t - nupd;
     const int i = k + 1 + tt / (k + 1), j = tt % (k + 1);
-    op.P = tile_at(p.Y, p.ld, j, k);
-    op.Q = tile_at(p.A, p.ld, i, k);
+    op.pm = kMapY, op.pr = j * kT, op.pc = k * kT;  // Y_jk
+    op.qm = kMapA, op.qr = i * kT, op.qc = k * kT;  // L_ik
     op.C = tile_at(p.Y, p.ld, j, i);
   }
   return op;
 }
 
-// The registers holding one chunk of both operands: thread t loads rows
-// t / 8 + 32 g (g < 4), 16 bytes at column 4 (t % 8) of the chunk.
-struct Chunk {
-  float4 p[4], q[4];
-};
-
-__device__ __forceinline__ void load_chunk(const TileOp& op, int c, Chunk& ch) {
-  const int cc = threadIdx.x & 7, r0 = threadIdx.x >> 3;
-#pragma unroll
-  for (int g = 0; g < 4; ++g) {
-    const int r = r0 + 32 * g;
-    ch.p[g] = __ldcg(reinterpret_cast<const float4*>(op.P + r * op.ldp + c * kCk + 4 * cc));
-    ch.q[g] = __ldcg(reinterpret_cast<const float4*>(op.Q + r * op.ldq + c * kCk + 4 * cc));
-  }
-}
-
 __device__ __forceinline__ float tf32_hi(float x) { return __uint_as_float(__float_as_uint(x) & 0xffffe000u); }
 
-__device__ __forceinline__ void put_split(uint8_t* hi, uint8_t* lo, uint32_t off, float4 v) {
-  const float4 h = make_float4(tf32_hi(v.x), tf32_hi(v.y), tf32_hi(v.z), tf32_hi(v.w));
-  *reinterpret_cast<float4*>(hi + off) = h;
-  *reinterpret_cast<float4*>(lo + off) = make_float4(v.x - h.x, v.y - h.y, v.z - h.z, v.w - h.w);
-}
-
-// Row r of a 128 x 32 fp32 operand chunk is one 128-byte row of the buffer
-// whose 16-byte pieces are permuted by XOR with (r mod 8): the layout a TMA
-// load with 128-byte swizzle writes, read by the MMA descriptors below.
-__device__ __forceinline__ void store_chunk(uint8_t* stage, const Chunk& ch) {
-  const int cc = threadIdx.x & 7, r0 = threadIdx.x >> 3;
+// lo = x - hi(x) for one chunk pair, elementwise (the layout is kept).
+__device__ __forceinline__ void form_lo(const uint8_t* raw, uint8_t* lo) {
 #pragma unroll
-  for (int g = 0; g < 4; ++g) {
-    const int r = r0 + 32 * g;
-    const uint32_t off = static_cast<uint32_t>(r * 128 + ((cc ^ (r & 7)) << 4));
-    put_split(stage, stage + kBufBytes, off, ch.p[g]);
-    put_split(stage + 2 * kBufBytes, stage + 3 * kBufBytes, off, ch.q[g]);
+  for (int u = 0; u < kPairBytes / 16 / kCholThreads; ++u) {
+    const int off = 16 * (threadIdx.x + u * kCholThreads);
+    const float4 x = *reinterpret_cast<const float4*>(raw + off);
+    *reinterpret_cast<float4*>(lo + off) =
+        make_float4(x.x - tf32_hi(x.x), x.y - tf32_hi(x.y), x.z - tf32_hi(x.z), x.w - tf32_hi(x.w));
   }
 }
 
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_all() { asm volatile("fence.proxy.async;" ::: "memory"); }
 
-// The three tf32 products of one staged chunk (4 K-steps of 8) into d_tmem.
-__device__ __forceinline__ void issue_chunk(const uint8_t* stage, uint32_t d_tmem, bool first) {
+// The three tf32 products of one chunk (4 K-steps of 8) into d_tmem: the raw
+// chunk read as the hi halves, the formed chunk as the lo halves.
+__device__ __forceinline__ void issue_chunk(const uint8_t* raw, const uint8_t* lo, uint32_t d_tmem, bool first) {
   const uint32_t idesc = instr_desc(2u, 0u, 0u, kT, kT);  // tf32, both operands K-major, 128 x 128
-  const uint32_t ph = smem_u32(stage), pl = ph + kBufBytes, qh = pl + kBufBytes, ql = qh + kBufBytes;
+  const uint32_t ph = smem_u32(raw), qh = ph + kBufBytes, pl = smem_u32(lo), ql = pl + kBufBytes;
 #pragma unroll
   for (int kk = 0; kk < kCk / 8; ++kk) {
     // K-major: the next 8 columns of K are 32 bytes further along each row
@@ -386,12 +373,15 @@ __device__ __forceinline__ void write_tile(const TileOp& op, int64_t ld, uint32_
 
 // Per-CTA pipeline state (identical in every thread).
 struct Pipe {
-  uint8_t* ring;         // kStages stages of kStageBytes, 1024-byte aligned
-  uint64_t* stage_free;  // [kStages]: completes when the MMAs reading a stage are done
-  uint64_t* acc_full;    // [2]: completes when an accumulator's products are done
+  uint8_t* raw;          // kRawStages chunk pairs as loaded, 1024-byte aligned
+  uint8_t* lo;           // kLoStages chunk pairs of low halves
+  uint64_t* raw_full;    // [kRawStages]: a chunk pair has landed
+  uint64_t* raw_free;    // [kRawStages]: the products reading a raw stage are done
+  uint64_t* lo_free;     // [kLoStages]: the products reading a lo stage are done
+  uint64_t* acc_full;    // [2]: an accumulator's products are done
   uint64_t* drain;
   uint32_t tmem;         // base of the two accumulators
-  uint32_t chunks;       // chunks staged so far (all phases)
+  uint32_t chunks;       // chunk pairs consumed so far (all phases)
   uint32_t ops;          // operations issued so far
 };
 
@@ -408,48 +398,92 @@ __device__ bool finish_op(const CholArgs& p, const Pipe& pp, const TileOp& op, u
   return true;
 }
 
+// Thread 0: the TMA loads of chunk c of `op` as chunk pair number q (its raw
+// stage must have been released by the products of pair q - kRawStages).
+__device__ __forceinline__ bool load_pair(const CholArgs& p, const Maps& mp, const Pipe& pp, const TileOp& op,
+                                          int c, uint32_t q) {
+  const uint32_t s = q % kRawStages;
+  if (q >= kRawStages && !mbar_wait(pp.raw_free + s, ((q - kRawStages) / kRawStages) & 1u, p.wait_ns)) return false;
+  uint8_t* dst = pp.raw + s * kPairBytes;
+  mbar_arrive_expect_tx(pp.raw_full + s, kPairBytes);
+  tma_load_2d(dst, mp.m[op.pm], pp.raw_full + s, op.pc + c * kCk, op.pr);
+  tma_load_2d(dst + kBufBytes, mp.m[op.qm], pp.raw_full + s, op.qc + c * kCk, op.qr);
+  return true;
+}
+
+// On a failure path, thread 0 waits (bounded) for the loads it issued but
+// nobody consumed, pairs [from, to) after `base`, so that no copy is still
+// landing in shared memory when the CTA returns.
+__device__ void drain_loads(const Pipe& pp, uint32_t base, int from, int to) {
+  if (threadIdx.x != 0) return;
+  for (int l = from; l < to; ++l) {
+    const uint32_t q = base + l;
+    mbar_wait(pp.raw_full + q % kRawStages, (q / kRawStages) & 1u, kDrainNs);
+  }
+}
+
+template <bool kPhaseU>
+__device__ __forceinline__ TileOp op_at(const CholArgs& p, int k, int t) {
+  return kPhaseU ? op_phase_u(p, k, t) : op_phase_t(p, k, t);
+}
+
 // Runs operations [lo, hi) of a phase.  Returns false if a wait ran out.
 // On return every product this CTA issued is done.
 template <bool kPhaseU>
-__device__ bool run_ops(const CholArgs& p, Pipe& pp, int k, int lo, int hi) {
+__device__ bool run_ops(const CholArgs& p, const Maps& mp, Pipe& pp, int k, int lo, int hi) {
   if (lo >= hi) return true;
-  Chunk ch;
-  TileOp cur = kPhaseU ? op_phase_u(p, k, lo) : op_phase_t(p, k, lo);
-  TileOp prev = cur;
-  load_chunk(cur, 0, ch);
-  for (int t = lo; t < hi; ++t) {
-    const bool more = t + 1 < hi;
-    const TileOp nxt = more ? (kPhaseU ? op_phase_u(p, k, t + 1) : op_phase_t(p, k, t + 1)) : cur;
-    const uint32_t buf = pp.ops & 1u;
+  const int npairs = (hi - lo) * kChunks;
+  const uint32_t base = pp.chunks;
+  // this CTA's earlier generic writes (the diagonal factor's shared memory,
+  // tiles written by its epilogues) before the TMA writes and reads below
+  fence_async_all();
+  __syncthreads();
+  int issued = 0;  // thread 0: pairs of this call whose loads are issued
+  bool ok0 = true;
+  if (threadIdx.x == 0) {
+    while (issued < kRawStages - 1 && issued < npairs && ok0) {
+      ok0 = load_pair(p, mp, pp, op_at<kPhaseU>(p, k, lo + issued / kChunks), issued % kChunks, base + issued);
+      if (ok0) ++issued;
+    }
+  }
+  TileOp cur = op_at<kPhaseU>(p, k, lo), prev = cur;
 #pragma unroll 1
-    for (int c = 0; c < kChunks; ++c) {
-      const uint32_t s = pp.chunks % kStages;
-      uint8_t* stage = pp.ring + s * kStageBytes;
-      bool ok = true;
-      if (pp.chunks >= kStages)  // the products that read this stage two chunks ago
-        ok = mbar_wait(pp.stage_free + s, ((pp.chunks - kStages) / kStages) & 1u, p.wait_ns);
-      if (ok) store_chunk(stage, ch);
-      if (c + 1 < kChunks)
-        load_chunk(cur, c + 1, ch);
-      else if (more)
-        load_chunk(nxt, 0, ch);
-      fence_async_smem();
-      if (!__syncthreads_and(ok)) {
-        give_up(p);
+  for (int l = 0; l < npairs; ++l) {
+    const int t = lo + l / kChunks, c = l % kChunks;
+    if (c == 0 && l > 0) cur = op_at<kPhaseU>(p, k, t);
+    const uint32_t q = base + l, s = q % kRawStages, s2 = q % kLoStages;
+    bool ok = mbar_wait(pp.raw_full + s, (q / kRawStages) & 1u, p.wait_ns);
+    if (ok && q >= kLoStages) ok = mbar_wait(pp.lo_free + s2, ((q - kLoStages) / kLoStages) & 1u, p.wait_ns);
+    const uint8_t* raw = pp.raw + s * kPairBytes;
+    uint8_t* lop = pp.lo + s2 * kPairBytes;
+    if (ok) form_lo(raw, lop);
+    fence_async_smem();
+    if (!__syncthreads_and(ok && ok0)) {
+      give_up(p);
+      drain_loads(pp, base, l + (ok ? 1 : 0), issued);
+      return false;
+    }
+    const uint32_t buf = pp.ops & 1u;
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      issue_chunk(raw, lop, pp.tmem + buf * kT, c == 0);
+      mma_commit(pp.raw_free + s);
+      mma_commit(pp.lo_free + s2);
+      if (c + 1 == kChunks) mma_commit(pp.acc_full + buf);
+      if (issued < npairs && ok0) {
+        ok0 = load_pair(p, mp, pp, op_at<kPhaseU>(p, k, lo + issued / kChunks), issued % kChunks, base + issued);
+        if (ok0) ++issued;
+      }
+    }
+    ++pp.chunks;
+    if (c + 1 == kChunks) {
+      if (t > lo && !finish_op(p, pp, prev, pp.ops - 1)) {
+        drain_loads(pp, base, l + 1, issued);
         return false;
       }
-      if (threadIdx.x == 0) {
-        tc_fence_after();
-        issue_chunk(stage, pp.tmem + buf * kT, c == 0);
-        mma_commit(pp.stage_free + s);
-        if (c + 1 == kChunks) mma_commit(pp.acc_full + buf);
-      }
-      ++pp.chunks;
+      prev = cur;
+      ++pp.ops;
     }
-    if (t > lo && !finish_op(p, pp, prev, pp.ops - 1)) return false;
-    prev = cur;
-    cur = nxt;
-    ++pp.ops;
   }
   return finish_op(p, pp, prev, pp.ops - 1);
 }
@@ -458,27 +492,36 @@ __device__ bool run_ops(const CholArgs& p, Pipe& pp, int k, int lo, int hi) {
 // row l / 2, columns 8 (l % 2) .. + 7 in v (only the lower half is read).
 // On return v holds L's lower half and rdiag[j] = 1 / L_jj.  A pivot that is
 // not positive or not finite raises a flag and is replaced by 1.
+//
+// At pivot j every lane subtracts (A_rj / A_jj) A_cj from each of its entries
+// right of column j (which of a lane's eight columns lie right of j is fixed
+// by j and the lane's half, so no lane branches); entries above the diagonal
+// take the same update and are never read.
 __device__ __forceinline__ void chol16(float (&v)[8], float* rdiag, bool& nonfinite, bool& notpd) {
   const int lane = threadIdx.x & 31, r = lane >> 1, h = lane & 1;
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
     const int jh = j >> 3, jq = j & 7;
-    float d = __shfl_sync(0xffffffffu, v[jq], 2 * j + jh);        // A_jj
-    const float mine = __shfl_sync(0xffffffffu, v[jq], 2 * r + jh);  // A_rj
+    float d = __shfl_sync(0xffffffffu, v[jq], 2 * j + jh);           // A_jj
+    const float mine = __shfl_sync(0xffffffffu, v[jq], 2 * r + jh);   // A_rj
     float col[8];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) col[q] = __shfl_sync(0xffffffffu, v[jq], 2 * (8 * h + q) + jh);  // A_cj
+    for (int q = 0; q < 8; ++q) col[q] = __shfl_sync(0xffffffffu, v[jq], 16 * h + 2 * q + jh);  // A_cj
     nonfinite |= !isfinite(d);
     notpd |= !(d > 0.0f);
     d = (d > 0.0f && d < INFINITY) ? d : 1.0f;
     const float rs = rsqrtf(d);
-    const float lr = mine * rs;  // L_rj
+    const float m = mine * (rs * rs);  // L_rj / L_jj
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-      const int c = 8 * h + q;
-      if (c > j && c <= r) v[q] = fmaf(-lr, col[q] * rs, v[q]);
+      if (q > j) {
+        v[q] = fmaf(-m, col[q], v[q]);  // column q (and 8 + q) right of j in both halves
+      } else if (q + 8 > j) {
+        const float u = fmaf(-m, col[q], v[q]);  // column 8 + q right of j: the upper half's lanes
+        v[q] = h ? u : v[q];
+      }
     }
-    if (h == jh) v[jq] = r > j ? lr : (r == j ? d * rs : v[jq]);
+    if (h == jh) v[jq] = r > j ? mine * rs : (r == j ? d * rs : v[jq]);
     if (lane == 0) rdiag[j] = rs;
   }
 }
@@ -572,10 +615,16 @@ __device__ void factor_block(const CholArgs& p, int k, float* fs) {
 #pragma unroll
       for (int c = 0; c < 16; ++c) XR[(b0 + c) * kSP + j] = x[c];
     }
-    __syncthreads();
-    if (e == kT) break;
-    // phase B
+    if (e == kT) {
+      __syncthreads();
+      break;
+    }
+    // phase B.  Warp 0 needs only the rows it solved itself (the 16 below the
+    // sub-panel), so it arrives at barrier 1 without waiting and starts on
+    // the next diagonal block; the other warps wait there for all of phase A.
     if (warp == 0) {
+      __syncwarp();
+      asm volatile("bar.arrive 1, %0;" ::"r"(kCholThreads) : "memory");
       const int r = lane >> 1, h = lane & 1, i = e + r, c0 = e + 8 * h;
       float v[8];
 #pragma unroll
@@ -598,6 +647,7 @@ __device__ void factor_block(const CholArgs& p, int k, float* fs) {
 #pragma unroll
       for (int q = 0; q < 8; ++q) S[i * kSP + c0 + q] = v[q];
     } else {
+      asm volatile("bar.sync 1, %0;" ::"r"(kCholThreads) : "memory");
       const int M4 = (kT - e) / 4, E4 = e / 4;
       const int ntr = M4 * (M4 + 1) / 2 - 10;  // lower 4 x 4 blocks outside warp 0's 16 x 16 block
       const int total = ntr + M4 * E4;
@@ -690,23 +740,35 @@ __device__ __forceinline__ void share(int total, int w, int workers, int& lo, in
   hi = static_cast<int>((static_cast<int64_t>(total) * (w + 1)) / workers);
 }
 
-__global__ void __launch_bounds__(kCholThreads, 1) chol_tc_kernel(CholArgs p) {
+__global__ void __launch_bounds__(kCholThreads, 1)
+    chol_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_y,
+                   const __grid_constant__ CUtensorMap map_l, CholArgs p) {
   extern __shared__ uint8_t chol_smem_raw[];
   uint8_t* region =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(chol_smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(region + kRegionBytes);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 6);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
   const int warp = threadIdx.x >> 5;
+  Maps mp;
+  mp.m[kMapA] = &map_a;
+  mp.m[kMapY] = &map_y;
+  mp.m[kMapL] = &map_l;
   Pipe pp;
-  pp.ring = region;
-  pp.stage_free = bars;
-  pp.acc_full = bars + 2;
-  pp.drain = bars + 4;
+  pp.raw = region;
+  pp.lo = region + static_cast<size_t>(kRawStages) * kPairBytes;
+  pp.raw_full = bars;
+  pp.raw_free = bars + kRawStages;
+  pp.lo_free = bars + 2 * kRawStages;
+  pp.acc_full = pp.lo_free + kLoStages;
+  pp.drain = pp.acc_full + 2;
   pp.chunks = 0;
   pp.ops = 0;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 5; ++i) mbar_init(bars + i, 1);
+    for (int i = 0; i < kNumBars; ++i) mbar_init(bars + i, 1);
     fence_barrier_init();
+    prefetch_tensormap(&map_a);
+    prefetch_tensormap(&map_y);
+    prefetch_tensormap(&map_l);
   }
   if (warp == 0) {
     tmem_alloc(tmem_slot, kCholTmemCols);
@@ -729,19 +791,19 @@ __global__ void __launch_bounds__(kCholThreads, 1) chol_tc_kernel(CholArgs p) {
     // inverse goes to the other Linv slot): the diagonal chain overlaps the
     // panel's products.
     if (G == 1) {
-      live = run_ops<false>(p, pp, k, 0, nb - 1);
+      live = run_ops<false>(p, mp, pp, k, 0, nb - 1);
     } else if (b == 0) {
-      live = run_ops<false>(p, pp, k, 0, m > 0 ? 1 : 0);
+      live = run_ops<false>(p, mp, pp, k, 0, m > 0 ? 1 : 0);
     } else {
       int lo, hi;
       share(nb - 1 - (m > 0 ? 1 : 0), b - 1, G - 1, lo, hi);
       const int off = m > 0 ? 1 : 0;
-      live = run_ops<false>(p, pp, k, off + lo, off + hi);
+      live = run_ops<false>(p, mp, pp, k, off + lo, off + hi);
     }
     if (!live) break;
     unsigned gen = grid_arrive(p);
     if (G > 1 && b == 0 && m > 0) {
-      live = run_ops<true>(p, pp, k, 0, 1);
+      live = run_ops<true>(p, mp, pp, k, 0, 1);
       __threadfence();
       __syncthreads();
       if (live) factor_block(p, k + 1, fs);
@@ -754,12 +816,12 @@ __global__ void __launch_bounds__(kCholThreads, 1) chol_tc_kernel(CholArgs p) {
     // CTAs other than CTA 0 (all of them when there is only one CTA).
     const int total = m * (m + 1) / 2 + m * (k + 1);
     if (G == 1) {
-      live = run_ops<true>(p, pp, k, 0, total);
+      live = run_ops<true>(p, mp, pp, k, 0, total);
       if (live && m > 0) factor_block(p, k + 1, fs);
     } else if (b > 0 && total > 1) {
       int lo, hi;
       share(total - 1, b - 1, G - 1, lo, hi);
-      live = run_ops<true>(p, pp, k, 1 + lo, 1 + hi);
+      live = run_ops<true>(p, mp, pp, k, 1 + lo, 1 + hi);
     }
     if (live) live = grid_sync(p);
   }
@@ -877,7 +939,13 @@ gptq_status prepare_hinv(const float* H, const double* hdiag, int n, float damp,
   ca.bar = bar;
   ca.abort = reinterpret_cast<int*>(bar + 2);
   ca.wait_ns = wait_limit_ns();
-  void* args[] = {&ca};
+  CUtensorMap map_a, map_y, map_l;
+  const CUtensorMapDataType f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  if (!make_tensor_map_2d(&map_a, f32, A, np, np, np * 4, kCk, kT, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tensor_map_2d(&map_y, f32, Y, np, np, np * 4, kCk, kT, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tensor_map_2d(&map_l, f32, ca.Linv, kT, 2 * kT, kT * 4, kCk, kT, CU_TENSOR_MAP_SWIZZLE_128B))
+    return GPTQ_ERR_CUDA;
+  void* args[] = {&map_a, &map_y, &map_l, &ca};
   const bool traced = trace_on();
   if (traced) trace_begin(st);
   if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(chol_tc_kernel), dim3(grid), dim3(kCholThreads), args,
