@@ -51,6 +51,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-gptq2d", action="store_true", help="skip the GPTQ-2D measurement")
     ap.add_argument("--no-others", action="store_true", help="skip the other synthetic workloads")
+    ap.add_argument("--profile-pass", action="store_true",
+                    help="no timing: two small layer passes (4096x4096, 32,768 tokens) and 8 packed matvecs, "
+                         "for kernel-by-kernel ncu captures")
     ap.add_argument("--cpu-tokens", type=int, default=4096, help="oracle sample: tokens for H")
     ap.add_argument("--cpu-rows", type=int, default=32, help="oracle sample: rows through the column loop")
     return ap.parse_args()
@@ -896,6 +899,11 @@ def run_e2e(args, spec, W, X, dev, world, dist):
     Wh = W.cpu().pin_memory()
     Xh = X.cpu().pin_memory()
     stream = torch.cuda.current_stream()
+    # the call allocates its own buffers through torch's caching allocator:
+    # start from an empty cache and warm it (two calls) so that no timed step
+    # waits on cudaMalloc / cudaFree
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
 
     def one():
         # host inputs straight into the public call: it streams X to the GPU in
@@ -906,6 +914,7 @@ def run_e2e(args, spec, W, X, dev, world, dist):
                out["scales"].to("cpu", non_blocking=True))
         return res
 
+    one()
     res = one()
     torch.cuda.synchronize()
     h2d = Wh.numel() * Wh.element_size() + Xh.numel() * Xh.element_size()
@@ -1047,8 +1056,33 @@ def run_reference(args, world, rank):
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def profile_pass():
+    """Two passes of the benchmark layer with an eighth of its tokens (the
+    factorization, column loop and packing see the full shapes; X is 268 MB,
+    larger than L2), then the packed-weight matvec 8 times: the command that
+    the ncu summaries under profiles/ capture, one kernel at a time."""
+    import torch
+
+    import post_weight_quantization_accum_b200 as gq
+    import synth_inputs as si
+
+    torch.cuda.set_device(0)
+    spec = si.scaled(si.SPECS["attn4096"], n_tok=32768)
+    W, X = si.make_layer(spec, "cuda")
+    for _ in range(2):
+        out = gq.quantize_layer(W, X, bits=spec.bits, group=spec.group, damp=spec.damp, block=spec.block)
+    x = torch.randn(spec.n, device="cuda").to(torch.bfloat16)
+    for _ in range(8):
+        gq.gptq_dequant_matvec(out["packed"], out["scales"], out["zeros"], spec.n, spec.bits, spec.group, x)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_pass": "ok", "kernel_launches": gq.gptq_kernel_launches()}))
+
+
 def main():
     args = parse_args()
+    if args.profile_pass:
+        profile_pass()
+        return
     world, rank, local = dist_env()
     if args.impl == "reference":
         res = run_reference(args, world, rank)

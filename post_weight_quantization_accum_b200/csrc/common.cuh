@@ -287,6 +287,43 @@ __device__ __forceinline__ void red_add_v4(float* dst, float4 v) {
                : "memory");
 }
 
+// A warp's 32 x 32 block of fp32 values (thread t holding row t in v) written
+// to dst (row pitch ld floats, 16-byte aligned rows) line by line: the block
+// goes through the warp's staging buffer stg (32 x 33 floats), and each
+// instruction then covers four rows with eight lanes per row, 128 contiguous
+// bytes each.  With sub, the values are subtracted as L2 reductions; without,
+// stored.  Valid rows are those below rows_left, valid columns below cols_left
+// (ragged edges of a matrix).  Rows and columns past them are not touched.
+__device__ __forceinline__ void warp_block_out(const uint32_t (&v)[32], float* stg, float* dst, int64_t ld, bool sub,
+                                               int rows_left, int cols_left, bool vec) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) stg[lane * 33 + j] = __uint_as_float(v[j]);
+  __syncwarp();
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int rr = 4 * it + (lane >> 3), cc = 4 * (lane & 7);
+    if (rr < rows_left && cc < cols_left) {
+      const float* s = stg + rr * 33 + cc;
+      float* d = dst + rr * ld + cc;
+      if (vec && cc + 4 <= cols_left) {
+        if (sub)
+          red_add_v4(d, make_float4(-s[0], -s[1], -s[2], -s[3]));
+        else
+          *reinterpret_cast<float4*>(d) = make_float4(s[0], s[1], s[2], s[3]);
+      } else {
+        for (int u = 0; u < 4 && cc + u < cols_left; ++u) {
+          if (sub)
+            atomicAdd(d + u, -s[u]);
+          else
+            d[u] = s[u];
+        }
+      }
+    }
+  }
+  __syncwarp();
+}
+
 // ---------------------------------------------------------------------------
 // host helpers
 // ---------------------------------------------------------------------------

@@ -152,7 +152,7 @@ __global__ void anti_transpose_kernel(const float* __restrict__ Y, int64_t ldy, 
 // its 13 low mantissa bits cleared, x_lo = x - x_hi; the dropped P_lo Q_lo is
 // below 2^-20 of the product).  The tensor cores read an fp32 operand as tf32
 // by dropping those 13 bits, so the chunks TMA brings in (128-byte swizzle,
-// K-major, a four-stage ring with three chunks in flight ahead) serve as the
+// K-major, a three-stage ring with two chunks in flight ahead) serve as the
 // hi halves as they are, and the threads only form the lo halves (a two-stage
 // ring in the same layout).  One thread issues the MMAs; the accumulator is
 // double-buffered, so one operation's epilogue (tensor memory -> registers ->
@@ -168,11 +168,12 @@ constexpr int kChunks = kT / kCk;
 constexpr int kCholThreads = 256;
 constexpr int kBufBytes = kT * kCk * 4;      // one 128 x 32 fp32 operand chunk (16 KB)
 constexpr int kPairBytes = 2 * kBufBytes;    // a chunk of both operands: P then Q
-constexpr int kRawStages = 4;                // operand chunks as loaded (TMA), 3 in flight ahead
+constexpr int kRawStages = 3;                // operand chunks as loaded (TMA), 2 in flight ahead
 constexpr int kLoStages = 2;                 // their low halves, formed by the threads
 constexpr int kSP = 132;                     // row pitch (floats) of the diagonal factor's matrices
 constexpr int kSub = 16;                     // sub-panel width of the diagonal factor
-constexpr size_t kRingBytes = static_cast<size_t>(kRawStages + kLoStages) * kPairBytes;
+constexpr size_t kStageFloats = 8 * 32 * 33;  // the epilogue's per-warp staging buffers
+constexpr size_t kRingBytes = static_cast<size_t>(kRawStages + kLoStages) * kPairBytes + kStageFloats * 4;
 constexpr size_t kFactorBytes = (2 * static_cast<size_t>(kT) * kSP + static_cast<size_t>(kSub) * kT + kT) * 4;
 constexpr size_t kRegionBytes = kFactorBytes > kRingBytes ? kFactorBytes : kRingBytes;
 constexpr int kNumBars = 2 * kRawStages + kLoStages + 2 + 1;  // raw full / free, lo free, accumulators, drain
@@ -347,27 +348,20 @@ __device__ __forceinline__ void issue_chunk(const uint8_t* raw, const uint8_t* l
 }
 
 // The accumulator into the output tile: warp w reads lanes 32 (w % 4) .. + 31
-// (tile rows) and columns 64 (w / 4) .. + 63, and stores them (or subtracts
-// them as L2 reductions, so the old values never travel to the SM).
-__device__ __forceinline__ void write_tile(const TileOp& op, int64_t ld, uint32_t acc) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+// (tile rows) and columns 64 (w / 4) .. + 63, and writes them row by row
+// through its staging buffer (whole 128-byte lines per four rows), as stores
+// or as L2 reductions (so the old values never travel to the SM).
+__device__ __forceinline__ void write_tile(const TileOp& op, int64_t ld, uint32_t acc, float* stage) {
+  const int warp = threadIdx.x >> 5;
   const int quad = warp & 3, half = warp >> 2;
-  float* row = op.C + static_cast<int64_t>(32 * quad + lane) * ld;
+  float* stg = stage + warp * 32 * 33;
 #pragma unroll
   for (int x = 0; x < 2; ++x) {
     const int c0 = 64 * half + 32 * x;
     uint32_t v[32];
     tmem_ld_32x32b_x32(acc + (static_cast<uint32_t>(32 * quad) << 16) + static_cast<uint32_t>(c0), v);
     tmem_ld_wait();
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const float4 f = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
-                                   __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
-      if (op.sub)
-        red_add_v4(row + c0 + 4 * q, make_float4(-f.x, -f.y, -f.z, -f.w));
-      else
-        *reinterpret_cast<float4*>(row + c0 + 4 * q) = f;
-    }
+    warp_block_out(v, stg, op.C + static_cast<int64_t>(32 * quad) * ld + c0, ld, op.sub != 0, 32, 32, true);
   }
 }
 
@@ -375,6 +369,7 @@ __device__ __forceinline__ void write_tile(const TileOp& op, int64_t ld, uint32_
 struct Pipe {
   uint8_t* raw;          // kRawStages chunk pairs as loaded, 1024-byte aligned
   uint8_t* lo;           // kLoStages chunk pairs of low halves
+  float* stage;          // [8 warps][32][33] epilogue staging
   uint64_t* raw_full;    // [kRawStages]: a chunk pair has landed
   uint64_t* raw_free;    // [kRawStages]: the products reading a raw stage are done
   uint64_t* lo_free;     // [kLoStages]: the products reading a lo stage are done
@@ -393,7 +388,7 @@ __device__ bool finish_op(const CholArgs& p, const Pipe& pp, const TileOp& op, u
     return false;
   }
   tc_fence_after();
-  write_tile(op, p.ld, pp.tmem + (o & 1u) * kT);
+  write_tile(op, p.ld, pp.tmem + (o & 1u) * kT, pp.stage);
   tc_fence_before();
   return true;
 }
@@ -756,6 +751,7 @@ __global__ void __launch_bounds__(kCholThreads, 1)
   Pipe pp;
   pp.raw = region;
   pp.lo = region + static_cast<size_t>(kRawStages) * kPairBytes;
+  pp.stage = reinterpret_cast<float*>(region + static_cast<size_t>(kRawStages + kLoStages) * kPairBytes);
   pp.raw_full = bars;
   pp.raw_free = bars + kRawStages;
   pp.lo_free = bars + 2 * kRawStages;

@@ -43,7 +43,8 @@ constexpr int kBBytes = kBN * kBK * 4;                  // 32 KB per split half 
 constexpr int kStageBytes = 2 * kABytes + 2 * kBBytes;  // 96 KB
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
-constexpr size_t kSmemBytes = 1024 + size_t(kStages) * kStageBytes + 256;
+constexpr size_t kStagingBytes = 4 * 32 * 33 * sizeof(float);  // the epilogue warps' staging buffers
+constexpr size_t kSmemBytes = 1024 + size_t(kStages) * kStageBytes + 256 + kStagingBytes;
 constexpr uint64_t kDrainNs = 2000000000ull;
 
 struct TrailParams {
@@ -71,6 +72,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* staging = reinterpret_cast<float*>(smem + size_t(kStages) * kStageBytes + 256);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -199,14 +201,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ---------------- epilogue: W -= accumulator ----------------
     const int quad = warp & 3;
-    const int r_in_tile = quad * 32 + lane;
     const bool vec = (p.ldw % 4 == 0) && (p.c0 % 4 == 0) && (reinterpret_cast<uintptr_t>(p.W) % 16 == 0);
     int local = 0;
     bool live = true;
     for (int t = blockIdx.x; t < num_tiles && live; t += gridDim.x)
     for (int u0 = 0; u0 < kchunks; u0 += p.unit_chunks, ++local) {
       const int tm = t / p.tiles_n, tn = t - tm * p.tiles_n;
-      const int row = tm * kBM + r_in_tile;
       const int col0 = p.c0 + tn * kBN;
       const int ncols = min(kBN, p.c0 + p.N - col0);
       const int buf = local & 1;
@@ -225,27 +225,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      float* wrow = p.W + static_cast<int64_t>(row) * p.ldw + col0;
+      // W -= acc as L2 reductions (nothing read back into the SM; each element
+      // receives one fp32 addition per launch, tiles being disjoint), written
+      // through the warp's staging buffer a whole 128-byte line at a time
+      float* stg = staging + (warp - 2) * 32 * 33;
+      const int row_base = tm * kBM + quad * 32;
+      float* wblk = p.W + static_cast<int64_t>(row_base) * p.ldw + col0;
       for (int c = 0; c < kBN; c += 32) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(buf * kBN + c), v);
         tmem_ld_wait();
-        if (row < p.M && c < ncols) {
-          // W -= acc as L2 reductions: nothing is read back into the SM, so
-          // the epilogue does not wait on L2 latency; each element receives
-          // one fp32 addition per launch (tiles are disjoint), the result of
-          // a load, an fp32 subtraction and a store
-          if (vec && c + 32 <= ncols) {
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-              red_add_v4(wrow + c + 4 * q, make_float4(-__uint_as_float(v[4 * q]), -__uint_as_float(v[4 * q + 1]),
-                                                       -__uint_as_float(v[4 * q + 2]), -__uint_as_float(v[4 * q + 3])));
-          } else {
-#pragma unroll
-            for (int q = 0; q < 32; ++q)
-              if (c + q < ncols) atomicAdd(wrow + c + q, -__uint_as_float(v[q]));
-          }
-        }
+        if (c < ncols && row_base < p.M)
+          warp_block_out(v, stg, wblk + c, p.ldw, true, p.M - row_base, ncols - c, vec);
       }
       tc_fence_before();
       __syncwarp();
