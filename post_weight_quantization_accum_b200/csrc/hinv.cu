@@ -143,8 +143,9 @@ __global__ void anti_transpose_kernel(const float* __restrict__ Y, int64_t ldy, 
 //               finalize  Y_jk   = Ry_jk Linv_kk^T          j < k
 //   phase U(k)  update    A_ij  -= L_ik L_jk^T              k < j <= i
 //               inverse   Ry_ji -= Y_jk L_ik^T              j <= k < i
-//               factor    Linv_{k+1,k+1} and Y_{k+1,k+1}    (CTA 0, right
-//                         after its own update of that tile)
+//               factor    Linv_{k+1,k+1}                     (CTA 0, right
+//                         after its own update of that tile; another CTA
+//                         writes Y_{k+1,k+1} = its transpose in phase T(k+1))
 //
 // Every operation is one 128 x 128 x 128 product on the tensor cores
 // (tcgen05.mma kind::tf32, fp32 accumulation in tensor memory), fp32-accurate
@@ -535,7 +536,7 @@ __device__ __forceinline__ void solve16(float (&x)[16], const float* S, const fl
 }
 
 // Factors the diagonal block k (by one CTA): Linv_kk into its Linv slot
-// (row-major) and Y_kk = Linv_kk^T into Y's diagonal tile.
+// (row-major).
 //
 // In 16-wide sub-panels s of the block S (its lower half), with R = I beside it:
 //   warp 0   Cholesky of the sub-panel's 16 x 16 diagonal block (chol16)
@@ -704,28 +705,40 @@ __device__ void factor_block(const CholArgs& p, int k, float* fs) {
     notpd = __any_sync(0xffffffffu, notpd);
     if (lane == 0 && (nonfinite || notpd)) set_status(p.fstatus, nonfinite ? GPTQ_ERR_NONFINITE : GPTQ_ERR_NOT_PD);
   }
-  // Linv (row-major, zeros above the diagonal); its transpose staged in S's
-  // place (conflict-free: consecutive threads take consecutive rows of X)
+  // Linv (row-major, zeros above the diagonal); Y_kk = Linv^T is written by
+  // another CTA from this slot (write_y_diag), off this CTA's chain
   for (int e = t; e < kT * (kT / 4); e += kCholThreads) {
     const int r = e >> 5, c = 4 * (e & 31);
     float4 x = *reinterpret_cast<const float4*>(XR + r * kSP + c);
     x = make_float4(c <= r ? x.x : 0.0f, c + 1 <= r ? x.y : 0.0f, c + 2 <= r ? x.z : 0.0f, c + 3 <= r ? x.w : 0.0f);
     *reinterpret_cast<float4*>(linv_slot(p, k) + r * kT + c) = x;
+  }
+  __threadfence();
+  __syncthreads();
+}
+
+// Y_kk = Linv_kk^T from Linv slot k % 2 (whole tile, zeros below the
+// diagonal), transposed through shared memory `T` ([kT][kSP] floats): reads
+// with consecutive threads on consecutive rows of Linv (conflict-free
+// transposed stores), then whole rows of Y written.
+__device__ void write_y_diag(const CholArgs& p, int k, float* T) {
+  const int t = threadIdx.x;
+  const float* L = linv_slot(p, k);
+  __syncthreads();
+  for (int e = t; e < kT * (kT / 4); e += kCholThreads) {
     const int rt = e & (kT - 1), ct = 4 * (e >> 7);
-    const float4 xt = *reinterpret_cast<const float4*>(XR + rt * kSP + ct);
-    S[ct * kSP + rt] = ct <= rt ? xt.x : 0.0f;
-    S[(ct + 1) * kSP + rt] = ct + 1 <= rt ? xt.y : 0.0f;
-    S[(ct + 2) * kSP + rt] = ct + 2 <= rt ? xt.z : 0.0f;
-    S[(ct + 3) * kSP + rt] = ct + 3 <= rt ? xt.w : 0.0f;
+    const float4 x = __ldcg(reinterpret_cast<const float4*>(L + rt * kT + ct));
+    T[ct * kSP + rt] = x.x;
+    T[(ct + 1) * kSP + rt] = x.y;
+    T[(ct + 2) * kSP + rt] = x.z;
+    T[(ct + 3) * kSP + rt] = x.w;
   }
   __syncthreads();
-  // Y_kk = Linv^T, row by row
   float* Ykk = tile_at(p.Y, p.ld, k, k);
   for (int e = t; e < kT * (kT / 4); e += kCholThreads) {
     const int r = e >> 5, c = 4 * (e & 31);
-    *reinterpret_cast<float4*>(Ykk + r * p.ld + c) = *reinterpret_cast<const float4*>(S + r * kSP + c);
+    *reinterpret_cast<float4*>(Ykk + r * p.ld + c) = *reinterpret_cast<const float4*>(T + r * kSP + c);
   }
-  __threadfence();
   __syncthreads();
 }
 
@@ -781,6 +794,9 @@ __global__ void __launch_bounds__(kCholThreads, 1)
   bool live = grid_sync(p);
   for (int k = 0; k < nb && live; ++k) {
     const int m = nb - 1 - k;
+    // Y_kk from the Linv slot written by the factor of block k (read from
+    // phase U(k) on), by the last CTA before its share of phase T(k)
+    if (b == G - 1) write_y_diag(p, k, fs);
     // Phase T(k).  CTA 0 takes the trsm of row block k+1 (operation 0), then
     // arrives, then, while the others finish the panel, updates tile
     // (k+1, k+1) with it (operation 0 of phase U) and factors block k+1 (its
