@@ -287,6 +287,12 @@ __device__ __forceinline__ void red_add_v4(float* dst, float4 v) {
                : "memory");
 }
 
+// Programmatic dependent launch: let the next kernel of the stream start
+// (its own pdl_wait holds it before dependent memory), and wait for every
+// earlier kernel of the stream to finish and flush its memory.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // A warp's 32 x 32 block of fp32 values (thread t holding row t in v) written
 // to dst (row pitch ld floats, 16-byte aligned rows) line by line: the block
 // goes through the warp's staging buffer stg (32 x 33 floats), and each
@@ -366,6 +372,32 @@ inline void launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
   kernel<<<grid, block, smem, st>>>(static_cast<KArgs>(args)...);
   if (traced) trace_end(st, reinterpret_cast<const void*>(kernel));
   count_launch();
+}
+
+// Launches `kernel` with programmatic stream serialization: it may start
+// while the previous kernel of the stream is still running, once every CTA of
+// that kernel has called pdl_trigger() (or exited).  The kernel must call
+// pdl_wait() before it touches any memory an earlier kernel of the stream
+// writes or reads.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const bool traced = trace_on();
+  if (traced) trace_begin(st);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+  if (traced) trace_end(st, reinterpret_cast<const void*>(kernel));
+  count_launch();
+  return e;
 }
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }

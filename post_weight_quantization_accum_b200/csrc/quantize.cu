@@ -118,6 +118,8 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32, 1) gptq_block_kernel(Blo
   const int lane = threadIdx.x & 31;
   const int li = lane % kLanes;  // lane within its row group
   const int warps = blockDim.x >> 5;
+  // the next kernel of the stream (a trailing update) may start its prologue
+  pdl_trigger();
   // the tile by asynchronous 4-byte copies, all in flight at once, scattered
   // to the lane-major layout (coalesced along U's rows; zeros outside the block)
   for (int e = threadIdx.x; e < kBMax * kBMax; e += blockDim.x) {
@@ -131,6 +133,9 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32, 1) gptq_block_kernel(Blo
   for (int j = threadIdx.x; j < kBMax; j += blockDim.x)
     rdiag[j] = j < bw ? 1.0f / us[j * Shape::kRowPitch + (j % kLanes) * Shape::kPitch + j / kLanes] : 0.0f;
   __syncthreads();
+  // U is fixed for the whole loop; everything below reads or writes what the
+  // previous kernels of the stream produce or consume (W, E, codes, groups)
+  pdl_wait();
 
   const int64_t warp_row0 = (static_cast<int64_t>(blockIdx.x) * warps + (threadIdx.x >> 5)) * (32 / kLanes);
   if (warp_row0 >= a.rows) return;  // whole warps leave; no block-wide barrier follows
@@ -438,7 +443,9 @@ gptq_status quantize_layer(const void* W, gptq_dtype wdt, int64_t rows, int n, c
                i1 + a.bw, gend, ext_minmax);
         a.ext_minmax = ext_minmax;
       }
-      launch(gptq_block_kernel<kBlockLanes>, block_ctas, warps_per_cta * 32, block_smem, st, a);
+      if (launch_pdl(gptq_block_kernel<kBlockLanes>, dim3(block_ctas), dim3(warps_per_cta * 32), block_smem, st, a) !=
+          cudaSuccess)
+        return GPTQ_ERR_CUDA;
       const int i2 = i1 + a.bw;
       if (i2 < s2) {  // inner update: the rest of the super-block
         const gptq_status ts = trailing_update_tc(Wk, n, static_cast<int>(rows), s2 - i2, a.bw, i2, i1, E_hi + a.e_off,

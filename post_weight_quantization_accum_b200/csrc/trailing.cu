@@ -97,6 +97,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
+  // the next kernel of the stream (a block kernel) may start its prologue;
+  // this one waits for the previous kernels before it reads E or touches W
+  pdl_trigger();
+  pdl_wait();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -332,8 +336,10 @@ gptq_status trailing_update_tc(float* W, int64_t ldw, int M, int N, int K, int c
   p.status = info->status;
   p.wait_ns = wait_limit_ns();
   const int grid = std::min(info->sm_count, p.tiles_m * p.tiles_n);
-  launch(trailing_tc_kernel, grid, kThreads, kSmemBytes, st, m_ehi, m_elo, m_uhi, m_ulo, p);
-  return launch_status();
+  if (launch_pdl(trailing_tc_kernel, dim3(grid), dim3(kThreads), kSmemBytes, st, m_ehi, m_elo, m_uhi, m_ulo, p) !=
+      cudaSuccess)
+    return GPTQ_ERR_CUDA;
+  return GPTQ_OK;
 }
 
 
