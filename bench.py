@@ -847,7 +847,7 @@ def measure_gptq2d(gq, dev, clocks, m=4096, n=4096, tokens=8192, reps=5, cpu_row
     achieved = flops / (ms * 1e-3) / 1e12
     res = {"workload": f"W {m}x{n} fp32 N(0, 0.02); HL, HR Grams of {tokens} N(0,1) tokens, damp 0.01; "
                        "scale 0.005, codes in [-8, 7]",
-            "kernels": "round2d_tile_kernel + push2d_kernel per tile wavefront",
+            "kernels": "round2d_tile_kernel (high-priority stream) + far_push_kernel (low-priority stream) per tile wavefront",
             "ms_per_call": ms, "launches_per_call": (gq.gptq_kernel_launches() - launches0) / reps,
             "weights_per_s": m * n / (ms * 1e-3),
             "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",

@@ -369,8 +369,11 @@ size_t gptq2d_workspace_size(int64_t m, int64_t n);
  *           W - Q = UL^T E UR and tr(HL (W - Q) HR (W - Q)^T) = sum e^2.
  *   ws      gptq2d_workspace_size(m, n) bytes, 256-byte aligned
  * Accumulates in fp32 on the CUDA cores; about 2 * (m + n) / 64 kernel
- * launches.  Asynchronous on `stream`.  Codes for non-finite inputs are
- * unspecified.
+ * launches, on two streams the library keeps per device (the tile rounds on a
+ * high-priority one, the pushes to tiles two or more wavefronts ahead on a
+ * low-priority one), joined to `stream` by events: asynchronous on `stream`;
+ * calls from several host threads on one device share those streams and run
+ * one after another.  Codes for non-finite inputs are unspecified.
  * Errors: GPTQ_ERR_INVALID_ARG (negative sizes or sizes above 4,194,304, a bad
  * dtype, scale or clamp range, NULL or misaligned pointers, small workspace),
  * before any launch; GPTQ_ERR_CUDA. */

@@ -81,8 +81,8 @@ def test_gptq2d_arguments_rejected_before_any_launch(lib):
     ws = lib.gptq2d_workspace_size
     ws.restype = ctypes.c_size_t
     ws.argtypes = [ctypes.c_int64, ctypes.c_int64]
-    assert ws(64, 64) == 3 * 64 * 64 * 4
-    assert ws(3, 5) == 3 * 256
+    assert ws(64, 64) == 5 * 64 * 64 * 4   # W copy, the far and near push buffers, E
+    assert ws(3, 5) == 5 * 256
     assert ws(-1, 5) == 0
     f = lib.gptq2d_round
     f.argtypes = [P, ctypes.c_int, ctypes.c_int64, ctypes.c_int64, P, P, ctypes.c_float, ctypes.c_int32,
