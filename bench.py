@@ -777,6 +777,11 @@ def measure_matvec(gq, packed, out, spec, dev, pk, copies=16, reps=64):
     for i in range(3):
         gq.gptq_dequant_matvec(mats[i], out["scales"], out["zeros"], n, spec.bits, spec.group, x, y=y)
     torch.cuda.synchronize()
+    gq.gptq_trace_read()  # which kernel the library dispatches for this shape
+    gq.gptq_trace_enable(True)
+    gq.gptq_dequant_matvec(mats[0], out["scales"], out["zeros"], n, spec.bits, spec.group, x, y=y)
+    kernel = ",".join(gq.gptq_trace_read()) or "unknown"
+    gq.gptq_trace_enable(False)
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         for i in range(reps):
@@ -794,7 +799,7 @@ def measure_matvec(gq, packed, out, spec, dev, pk, copies=16, reps=64):
     del graph
     nbytes = packed.numel() * 4 + rows * ng * 5 + n * 2 + rows * 4
     gbs = nbytes / (us * 1e-6) / 1e9
-    return {"kernel": "dequant_matvec_kernel", "batch": 1, "us_per_call": us,
+    return {"kernel": kernel, "batch": 1, "us_per_call": us,
             "algorithmic_bytes": nbytes, "achieved_gbs": gbs, "peak_gbs": pk["hbm_gbs"],
             "frac": gbs / pk["hbm_gbs"], "bf16_equivalent_us_at_peak": rows * n * 2 / pk["hbm_gbs"] / 1e3}
 

@@ -21,7 +21,10 @@ if torch.cuda.is_available():
     import post_weight_quantization_accum_b200 as gq
 
 
-def _case(rows, n, bits, group, batch, act_order, xdtype, seed):
+def _case(rows, n, bits, group, batch, act_order, xdtype, seed, offset=0, zero_codes=False):
+    """`offset` widens the bound's magnitude for kernels that round
+    s * (offset + code) * x terms (the tensor-core path: offset 256 covers both
+    its 128 + code and 128 + z terms)."""
     rng = np.random.default_rng(seed)
     maxq = (1 << bits) - 1
     G = group if group > 0 else n
@@ -29,6 +32,9 @@ def _case(rows, n, bits, group, batch, act_order, xdtype, seed):
     codes = rng.integers(0, maxq + 1, size=(rows, n))
     scales = rng.uniform(0.001, 0.02, size=(rows, ng)).astype(np.float32)
     zeros = rng.integers(0, maxq + 1, size=(rows, ng))
+    if zero_codes:
+        codes[:] = 0
+        zeros[:] = 0
     g_idx = rng.permutation(np.arange(n) // G) if act_order else None
     x = rng.standard_normal((batch, n)).astype(np.float32)
     if xdtype == torch.bfloat16:
@@ -42,8 +48,8 @@ def _case(rows, n, bits, group, batch, act_order, xdtype, seed):
     torch.cuda.synchronize()
     ref = go.dequant_matvec(packed, scales, zeros, n, bits, group, x, g_idx)
     g = g_idx if g_idx is not None else np.arange(n) // G
-    mag = np.abs(scales.astype(np.float64)[:, g]) * (codes + zeros[:, g])  # [rows, n]: |s| (|code| + |z|)
-    bound = 5e-5 * (np.abs(x.astype(np.float64)) @ mag.T)
+    mag = np.abs(scales.astype(np.float64)[:, g]) * (offset + codes + zeros[:, g])  # |s| (offset + |code| + |z|)
+    bound = (4e-6 if offset else 5e-5) * (np.abs(x.astype(np.float64)) @ mag.T)
     return y.double().cpu().numpy(), ref, bound
 
 
@@ -58,6 +64,33 @@ def test_matvec_matches_oracle(bits, group):
 def test_matvec_batched_bf16_inputs(batch):
     y, ref, bound = _case(64, 1024, 4, 128, batch, False, torch.bfloat16, batch)
     assert y.shape == ref.shape
+    assert np.all(np.abs(y - ref) <= bound)
+
+
+@pytest.mark.parametrize("rows,n,group,batch", [
+    (1, 128, 0, 1), (37, 512, 0, 1), (100, 512, 32, 1), (64, 1024, 64, 5), (48, 2048, 256, 2),
+    (20, 512, 384, 3), (17, 4096, 0, 8), (33, 9216, 128, 1), (64, 11008, 128, 4), (16, 16384, 128, 8),
+    (4096, 4096, 128, 1)])
+def test_matvec_tensor_core_path(rows, n, group, batch):
+    """4-bit codes and bf16 x with n % 128 == 0: groups of a multiple of 128
+    columns (or one group per row) take the mma.sync path (16-row tiles,
+    128-column blocks, 4 blocks per warp and round, so n = 9216, 11008 and
+    16384 take several rounds), groups of 32 and 64 the general kernel.
+    Error of the mma.sync path: per block the fp32 sum of s (128 + code) x
+    over 8 chained MMAs (each adding 16 exact products), then the warp's
+    blocks (n / 1024) and the 8 warps in sequence, minus the offsets
+    sum_q s (128 + z) X_q (X_q from 8-value sums in 16- and T-lane trees):
+    at most ~(8 + n / 1024 + 8 + 12) eps sum |s| (256 + code + z) |x|
+    <= 2.7e-6 of that sum for n <= 16384; the bar is 4e-6."""
+    y, ref, bound = _case(rows, n, 4, group, batch, False, torch.bfloat16, rows + n + batch, offset=256)
+    assert y.shape == ref.shape
+    assert np.all(np.abs(y - ref) <= bound)
+
+
+def test_matvec_tensor_core_path_zero_codes():
+    # every code and zero point 0: the 128 offsets cancel to rounding noise
+    y, ref, bound = _case(40, 1024, 4, 128, 2, False, torch.bfloat16, 5, offset=256, zero_codes=True)
+    assert np.all(ref == 0)
     assert np.all(np.abs(y - ref) <= bound)
 
 
