@@ -532,6 +532,7 @@ def run_ours(args, world, rank, local):
     result["stage_rooflines"] = stage_rooflines(
         dict(zip(("hessian", "prepare_hinv", "quantize_layer", "pack"), stage_ms)), rows, n, spec.bits, ng, pk)
     result["packed_matvec"] = measure_matvec(gq, packed, out, spec, dev, pk)
+    result["column_loops"] = measure_column_loops(gq, lp)
     if not args.no_gptq2d:
         cpu_rows = 64 if (world == 1 and rank == 0 and not args.no_cpu_baseline) else 0
         result["gptq2d"] = measure_gptq2d(gq, dev, result.get("clocks"), cpu_rows=cpu_rows)
@@ -759,6 +760,49 @@ def run_layerset(args, world, rank, local):
         dist.barrier()
         dist.destroy_process_group()
     return result if rank == 0 else None
+
+
+def measure_column_loops(gq, lp, reps=10):
+    """The column loop (gptq_quantize_layer on the layer's U) timed with each
+    loop of gptq_set_column_loop: 0 per-block kernels (the default, the one
+    the step times), 1 the fused row-slab pass; and how many codes the two
+    share.  Outside the timed step."""
+    import torch
+
+    spec, st = lp.spec, lp.stream
+    res = {}
+    codes = {}
+    try:
+        for mode, name in ((0, "per_block"), (1, "fused_row_slab")):
+            gq.gptq_set_column_loop(mode)
+
+            def run():
+                gq.gptq_quantize_layer(lp.W, lp.U, spec.bits, spec.group, spec.block,
+                                       perm=lp.perm if spec.act_order else None, dead=lp.dead, out=lp.out, ws=lp.ws_q)
+
+            for _ in range(3):
+                run()
+            torch.cuda.synchronize()
+            codes[name] = lp.out["codes"].clone()
+            s = torch.cuda.Event(enable_timing=True)
+            e = torch.cuda.Event(enable_timing=True)
+            s.record(st)
+            for _ in range(reps):
+                run()
+            e.record(st)
+            torch.cuda.synchronize()
+            gq.gptq_trace_read()
+            gq.gptq_trace_enable(True)
+            run()
+            torch.cuda.synchronize()
+            trace = gq.gptq_trace_read()
+            gq.gptq_trace_enable(False)
+            res[name] = {"ms": s.elapsed_time(e) / reps,
+                         "kernels": {k: {"launches": v[0], "ms": v[1]} for k, v in trace.items()}}
+    finally:
+        gq.gptq_set_column_loop(0)
+    res["codes_agree"] = float((codes["per_block"] == codes["fused_row_slab"]).float().mean())
+    return res
 
 
 def measure_matvec(gq, packed, out, spec, dev, pk, copies=16, reps=64):

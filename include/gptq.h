@@ -121,6 +121,24 @@ int32_t gptq_trace_read(gptq_trace_entry* out, int32_t max_entries);
  * satisfied give up. */
 void gptq_set_wait_limit_ns(uint64_t ns);
 
+/* Column loop of gptq_quantize_layer (process-wide, read at each call, safe
+ * to set from any thread; GPTQ knowledge note, "How It Works": 128-column
+ * blocks whose corrections accumulate before one global update).
+ *   0 (default): per block, one quantize-and-propagate kernel over all rows
+ *      and one tensor-core update of the rest of its 1024-column super-block,
+ *      chained by programmatic dependent launch; one update per super-block
+ *      for the rest of the matrix.
+ *   1: the fused single pass per row slab: one launch per super-block in
+ *      which each CTA takes its rows through all of the super-block's blocks,
+ *      applying the earlier blocks' corrections left-looking (fp32, CUDA
+ *      cores) before each block's chain; the same outer updates.  Used where
+ *      it applies (n >= 2048, block 128, groups that divide 128 or one group
+ *      per row, at most 32 rows per SM), the default loop elsewhere.  Same
+ *      sums in another order: codes agree with mode 0 to fp32 rounding.
+ * Other values select 0. */
+void gptq_set_column_loop(int32_t mode);
+int32_t gptq_get_column_loop(void);
+
 /* ------------------------------------------------------------------------ */
 /* 1. Hessian accumulation                                                   */
 /* ------------------------------------------------------------------------ */

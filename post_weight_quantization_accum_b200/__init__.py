@@ -25,6 +25,8 @@ __all__ = [
     "gptq2d_factor",
     "gptq_get_device_status",
     "gptq_set_wait_limit_ns",
+    "gptq_set_column_loop",
+    "gptq_get_column_loop",
     "gptq_kernel_launches",
     "gptq_trace_enable",
     "gptq_trace_read",
@@ -67,6 +69,15 @@ def gptq_get_device_status(stream=None):
 
 def gptq_set_wait_limit_ns(ns):
     LIB.gptq_set_wait_limit_ns(ctypes.c_uint64(ns))
+
+
+def gptq_set_column_loop(mode):
+    """0: per-block kernels (default); 1: the fused row-slab pass where it applies."""
+    LIB.gptq_set_column_loop(int(mode))
+
+
+def gptq_get_column_loop():
+    return int(LIB.gptq_get_column_loop())
 
 
 def gptq_kernel_launches():

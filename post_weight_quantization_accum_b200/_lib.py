@@ -31,6 +31,8 @@ _SIGS = {
     "gptq_kernel_launches": (ctypes.c_uint64, []),
     "gptq_get_device_status": (ctypes.c_int, [_P]),
     "gptq_set_wait_limit_ns": (None, [ctypes.c_uint64]),
+    "gptq_set_column_loop": (None, [ctypes.c_int32]),
+    "gptq_get_column_loop": (ctypes.c_int32, []),
     "gptq_trace_enable": (None, [ctypes.c_int32]),
     "gptq_trace_read": (ctypes.c_int32, [_P, ctypes.c_int32]),
     "gptq_hessian_workspace_size": (ctypes.c_size_t, [ctypes.c_int32, ctypes.c_int64]),

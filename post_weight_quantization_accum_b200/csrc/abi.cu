@@ -108,6 +108,9 @@ bool make_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void*
 
 uint64_t wait_limit_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
 
+static std::atomic<int> g_column_loop{0};  // gptq_set_column_loop
+int column_loop_mode() { return g_column_loop.load(std::memory_order_relaxed); }
+
 static std::atomic<uint64_t> g_launches{0};
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
@@ -227,6 +230,10 @@ const char* gptq_status_string(gptq_status s) {
 int32_t gptq_version(void) { return 100; }
 
 uint64_t gptq_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+void gptq_set_column_loop(int32_t mode) { gptq::g_column_loop.store(mode == 1 ? 1 : 0, std::memory_order_relaxed); }
+
+int32_t gptq_get_column_loop(void) { return gptq::column_loop_mode(); }
 
 void gptq_set_wait_limit_ns(uint64_t ns) {
   g_wait_ns.store(ns == UINT64_MAX ? kDefaultWaitNs : ns, std::memory_order_relaxed);

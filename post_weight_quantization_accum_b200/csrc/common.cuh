@@ -87,6 +87,13 @@ __device__ __forceinline__ void cp_async_4(void* smem_dst, const void* gmem_src,
                : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
+// Closes the group of this thread's cp.async copies issued since the last
+// commit; cp_async_wait_group<N> waits until at most N groups are pending.
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
 
 // TMA (cp.async.bulk.tensor), no multicast
 // ---------------------------------------------------------------------------
@@ -350,6 +357,9 @@ bool make_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void*
 
 // Wait limit for pipeline barriers in nanoseconds (tests may shorten it).
 uint64_t wait_limit_ns();
+
+// Column loop selected by gptq_set_column_loop (0 per block, 1 fused).
+int column_loop_mode();
 
 inline gptq_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;

@@ -26,6 +26,9 @@
 //                       on the tensor cores, fp32-accurate through a 3-term
 //                       tf32 split; the block kernel writes E as its tf32
 //                       hi / lo halves.
+// gptq_superblock_kernel (selected by gptq_set_column_loop(1)) is the fused
+// single pass: one launch per super-block in which each CTA takes a slab of
+// rows through all of the super-block's blocks (described at the kernel).
 #include <algorithm>
 #include <atomic>
 #include <cstring>
@@ -107,48 +110,33 @@ struct BlockShape {
   static constexpr size_t kSmem = (static_cast<size_t>(kBMax) * kRowPitch + kBMax) * sizeof(float);
 };
 
+// The U tile rows [j0, j0 + nr) x columns [c0, c0 + nc) into the lane-major
+// layout by asynchronous 4-byte copies, all in flight at once (coalesced
+// along U's rows; zeros outside the tile's extent).  The caller waits.
 template <int kLanes>
-__global__ void __launch_bounds__(kMaxWarpsPerCta * 32, 1) gptq_block_kernel(BlockArgs a) {
+__device__ __forceinline__ void stage_u_tile(float* us, const float* __restrict__ U, int n, int j0, int c0, int nr,
+                                             int nc) {
   using Shape = BlockShape<kLanes>;
-  constexpr int C = Shape::kCols;
-  extern __shared__ __align__(16) float dyn_smem[];
-  float* us = dyn_smem;                             // [kBMax][kRowPitch] the U tile, lane-major
-  float* rdiag = us + kBMax * Shape::kRowPitch;     // [kBMax] 1 / U_jj
-  const int bw = a.bw;
-  const int lane = threadIdx.x & 31;
-  const int li = lane % kLanes;  // lane within its row group
-  const int warps = blockDim.x >> 5;
-  // the next kernel of the stream (a trailing update) may start its prologue
-  pdl_trigger();
-  // the tile by asynchronous 4-byte copies, all in flight at once, scattered
-  // to the lane-major layout (coalesced along U's rows; zeros outside the block)
   for (int e = threadIdx.x; e < kBMax * kBMax; e += blockDim.x) {
     const int j = e / kBMax, c = e % kBMax;
-    const bool in = j < bw && c < bw;
-    const float* src = in ? a.U + static_cast<int64_t>(a.i1 + j) * a.n + a.i1 + c : a.U;
+    const bool in = j < nr && c < nc;
+    const float* src = in ? U + static_cast<int64_t>(j0 + j) * n + c0 + c : U;
     cp_async_4(us + j * Shape::kRowPitch + (c % kLanes) * Shape::kPitch + c / kLanes, src, in ? 4u : 0u);
   }
-  cp_async_wait_all();
-  __syncthreads();
-  for (int j = threadIdx.x; j < kBMax; j += blockDim.x)
-    rdiag[j] = j < bw ? 1.0f / us[j * Shape::kRowPitch + (j % kLanes) * Shape::kPitch + j / kLanes] : 0.0f;
-  __syncthreads();
-  // U is fixed for the whole loop; everything below reads or writes what the
-  // previous kernels of the stream produce or consume (W, E, codes, groups)
-  pdl_wait();
+}
 
-  const int64_t warp_row0 = (static_cast<int64_t>(blockIdx.x) * warps + (threadIdx.x >> 5)) * (32 / kLanes);
-  if (warp_row0 >= a.rows) return;  // whole warps leave; no block-wide barrier follows
-  const int64_t r = warp_row0 + lane / kLanes;
-  const bool valid = r < a.rows;    // a warp's last rows may lie past the matrix
-  const int64_t rr = valid ? r : a.rows - 1;  // such lanes compute on a real row and write nothing
-  const float* wsrc = a.Wk + rr * a.n + a.i1;
-  float w[C];
-#pragma unroll
-  for (int m = 0; m < C; ++m) {
-    const int c = li + kLanes * m;
-    w[m] = c < bw ? wsrc[c] : 0.0f;
-  }
+// One row's quantize-and-propagate chain over the block [a.i1, a.i1 + a.bw):
+// w holds the lane's columns li + kLanes m of the block (fully updated by
+// every earlier column), us the block's diagonal U tile and rdiag 1 / U_jj.
+// Writes the row's codes, group parameters, scaled errors (tf32 hi / lo) and
+// loss; lanes of rows past the matrix (valid false) compute on row rr and
+// write nothing.
+template <int kLanes>
+__device__ __forceinline__ void block_chain(const BlockArgs& a, const float* us, const float* rdiag, int64_t r,
+                                            bool valid, int64_t rr, int li, float (&w)[BlockShape<kLanes>::kCols]) {
+  using Shape = BlockShape<kLanes>;
+  constexpr int C = Shape::kCols;
+  const int bw = a.bw;
   // A group that began in an earlier block keeps the (scale, zero) that
   // block fixed; they are read back from the outputs.
   GridParams gp{1.0f, 0.0f};
@@ -238,6 +226,158 @@ __global__ void __launch_bounds__(kMaxWarpsPerCta * 32, 1) gptq_block_kernel(Blo
     }
   }
   if (li == 0 && a.row_loss != nullptr) a.row_loss[r] += loss;
+}
+
+template <int kLanes>
+__global__ void __launch_bounds__(kMaxWarpsPerCta * 32, 1) gptq_block_kernel(BlockArgs a) {
+  using Shape = BlockShape<kLanes>;
+  constexpr int C = Shape::kCols;
+  extern __shared__ __align__(16) float dyn_smem[];
+  float* us = dyn_smem;                             // [kBMax][kRowPitch] the U tile, lane-major
+  float* rdiag = us + kBMax * Shape::kRowPitch;     // [kBMax] 1 / U_jj
+  const int bw = a.bw;
+  const int lane = threadIdx.x & 31;
+  const int li = lane % kLanes;  // lane within its row group
+  const int warps = blockDim.x >> 5;
+  // the next kernel of the stream (a trailing update) may start its prologue
+  pdl_trigger();
+  stage_u_tile<kLanes>(us, a.U, a.n, a.i1, a.i1, bw, bw);
+  cp_async_wait_all();
+  __syncthreads();
+  for (int j = threadIdx.x; j < kBMax; j += blockDim.x)
+    rdiag[j] = j < bw ? 1.0f / us[j * Shape::kRowPitch + (j % kLanes) * Shape::kPitch + j / kLanes] : 0.0f;
+  __syncthreads();
+  // U is fixed for the whole loop; everything below reads or writes what the
+  // previous kernels of the stream produce or consume (W, E, codes, groups)
+  pdl_wait();
+
+  const int64_t warp_row0 = (static_cast<int64_t>(blockIdx.x) * warps + (threadIdx.x >> 5)) * (32 / kLanes);
+  if (warp_row0 >= a.rows) return;  // whole warps leave; no block-wide barrier follows
+  const int64_t r = warp_row0 + lane / kLanes;
+  const bool valid = r < a.rows;    // a warp's last rows may lie past the matrix
+  const int64_t rr = valid ? r : a.rows - 1;  // such lanes compute on a real row and write nothing
+  const float* wsrc = a.Wk + rr * a.n + a.i1;
+  float w[C];
+#pragma unroll
+  for (int m = 0; m < C; ++m) {
+    const int c = li + kLanes * m;
+    w[m] = c < bw ? wsrc[c] : 0.0f;
+  }
+  block_chain<kLanes>(a, us, rdiag, r, valid, rr, li, w);
+}
+
+// One launch per super-block [s1, s2) (fused single pass over a row slab):
+// a CTA takes rows_cta = blockDim.x / kLanes rows through every block of the
+// super-block.  Block i1 starts from the rows' working weights as the
+// previous super-blocks left them and first applies, left-looking, the
+// corrections of the super-block's earlier blocks t: w_c -= sum_k E_t[r, k]
+// U[t + k, c] over this lane's columns c, fp32 on the CUDA cores, with the
+// U tiles (128 x 128) double-buffered in shared memory and the CTA's own
+// error rows read back from L2; then the block's chain runs as in
+// gptq_block_kernel.  The same sums as the per-block trailing updates in
+// another order (every column still receives every earlier column's
+// correction before it is quantized).  Requires that no group starting in a
+// later block of the super-block reaches past its block (block % G == 0, or
+// one group per row): a group's parameters need its columns' current values,
+// which the left-looking form has only for the block at hand.  ext_minmax
+// belongs to the first block.
+constexpr int kSlabMaxRows = 32;  // rows per CTA of the fused kernel (one CTA per SM)
+
+template <int kLanes>
+__global__ void __launch_bounds__(kSlabMaxRows * kLanes, 1) gptq_superblock_kernel(BlockArgs a, int s1, int s2,
+                                                                                   int block) {
+  using Shape = BlockShape<kLanes>;
+  constexpr int C = Shape::kCols;
+  constexpr int kTile = kBMax * Shape::kRowPitch;
+  extern __shared__ __align__(16) float dyn_smem[];
+  float* ubuf0 = dyn_smem;             // U tiles, lane-major, two buffers
+  float* ubuf1 = dyn_smem + kTile;
+  float* rdiag = ubuf1 + kTile;        // [kBMax] 1 / U_jj of the block at hand
+  const int lane = threadIdx.x & 31;
+  const int li = lane % kLanes;
+  const int rows_cta = blockDim.x / kLanes;
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * rows_cta + threadIdx.x / kLanes;
+  const bool valid = r < a.rows;
+  const int64_t rr = valid ? r : a.rows - 1;  // such lanes compute on a real row and write nothing
+  for (int i1 = s1; i1 < s2; i1 += block) {
+    BlockArgs b = a;
+    b.i1 = i1;
+    b.bw = min(block, s2 - i1);
+    b.e_off = i1 - s1;
+    if (i1 != s1) b.ext_minmax = nullptr;
+    const int bw = b.bw;
+    float w[C];
+    const float* wsrc = a.Wk + rr * a.n + i1;
+#pragma unroll
+    for (int m = 0; m < C; ++m) {
+      const int c = li + kLanes * m;
+      w[m] = c < bw ? wsrc[c] : 0.0f;
+    }
+    const int nt = (i1 - s1) / block;  // earlier blocks of the super-block, all `block` wide
+    if (nt > 0) {
+      // E of block t for this row (written earlier in this launch: plain L2
+      // loads, not the read-only path), e = hi + lo exactly: lane li keeps
+      // k = 8 li .. 8 li + 7 and hands them to its row's lanes by shuffle;
+      // the next tile's values are requested before this tile is used
+      auto load_e = [&](int t, float (&e)[8]) {
+        const float4* eh = reinterpret_cast<const float4*>(a.E_hi + rr * a.lde + t * block + 8 * li);
+        const float4* el = reinterpret_cast<const float4*>(a.E_lo + rr * a.lde + t * block + 8 * li);
+        const float4 h0 = __ldcg(eh), h1 = __ldcg(eh + 1), l0 = __ldcg(el), l1 = __ldcg(el + 1);
+        e[0] = h0.x + l0.x;
+        e[1] = h0.y + l0.y;
+        e[2] = h0.z + l0.z;
+        e[3] = h0.w + l0.w;
+        e[4] = h1.x + l1.x;
+        e[5] = h1.y + l1.y;
+        e[6] = h1.z + l1.z;
+        e[7] = h1.w + l1.w;
+      };
+      float e_cur[8], e_next[8];
+      load_e(0, e_cur);
+      stage_u_tile<kLanes>(ubuf0, a.U, a.n, s1, i1, block, bw);
+      cp_async_commit();
+      for (int t = 0; t < nt; ++t) {
+        const float* cur = (t & 1) ? ubuf1 : ubuf0;
+        if (t + 1 < nt) {
+          load_e(t + 1, e_next);
+          stage_u_tile<kLanes>((t & 1) ? ubuf0 : ubuf1, a.U, a.n, s1 + (t + 1) * block, i1, block, bw);
+          cp_async_commit();
+          cp_async_wait_group<1>();
+        } else {
+          cp_async_wait_group<0>();
+        }
+        __syncthreads();
+        const float* ulane = cur + li * Shape::kPitch;
+#pragma unroll 1
+        for (int kb = 0; kb < kBMax / 8; ++kb) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const float e = __shfl_sync(0xffffffffu, e_cur[kk], kb, kLanes);
+            const float4* urow = reinterpret_cast<const float4*>(ulane + (8 * kb + kk) * Shape::kRowPitch);
+#pragma unroll
+            for (int g4 = 0; g4 < C / 4; ++g4) {
+              const float4 u = urow[g4];
+              w[4 * g4 + 0] = fmaf(-e, u.x, w[4 * g4 + 0]);
+              w[4 * g4 + 1] = fmaf(-e, u.y, w[4 * g4 + 1]);
+              w[4 * g4 + 2] = fmaf(-e, u.z, w[4 * g4 + 2]);
+              w[4 * g4 + 3] = fmaf(-e, u.w, w[4 * g4 + 3]);
+            }
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) e_cur[i] = e_next[i];
+        __syncthreads();  // the buffer is refilled by a later tile
+      }
+    }
+    stage_u_tile<kLanes>(ubuf0, a.U, a.n, i1, i1, bw, bw);
+    cp_async_wait_all();
+    __syncthreads();
+    for (int j = threadIdx.x; j < kBMax; j += blockDim.x)
+      rdiag[j] = j < bw ? 1.0f / ubuf0[j * Shape::kRowPitch + (j % kLanes) * Shape::kPitch + j / kLanes] : 0.0f;
+    __syncthreads();
+    block_chain<kLanes>(b, ubuf0, rdiag, r, valid, rr, li, w);
+    __syncthreads();  // this block's errors are visible to the CTA; the tile buffer is free
+  }
 }
 
 // Per row, (min, max) of Wk[r, c0 : c1): the part of a group that lies past
@@ -428,9 +568,38 @@ gptq_status quantize_layer(const void* W, gptq_dtype wdt, int64_t rows, int n, c
     attr_set[info->device] = true;
   }
   const int S = super_width(l, n, block, G);
+  // Fused single pass (gptq_set_column_loop(1)) where it applies: a
+  // two-level loop with 128-wide blocks whose groups stay inside one block
+  // (or one group per row), and rows that fit one slab of at most
+  // kSlabMaxRows per SM: one launch per super-block.
+  const int64_t slab = 2 * ceil_div(rows, 2 * static_cast<int64_t>(info->sm_count));
+  const bool fused = column_loop_mode() == 1 && S > block && block == kBMax && (block % G == 0 || G == n) &&
+                     slab <= kSlabMaxRows;
+  constexpr size_t super_smem = (2 * static_cast<size_t>(kBMax) * BlockShape<kBlockLanes>::kRowPitch + kBMax) * sizeof(float);
+  const int rows_cta = static_cast<int>(std::max<int64_t>(2, slab));
+  if (fused) {
+    static std::atomic<bool> super_attr[64] = {};
+    if (!super_attr[info->device]) {
+      if (cudaFuncSetAttribute(gptq_superblock_kernel<kBlockLanes>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(super_smem)) != cudaSuccess)
+        return GPTQ_ERR_CUDA;
+      super_attr[info->device] = true;
+    }
+  }
   for (int s1 = 0; s1 < n; s1 += S) {
     const int s2 = std::min(s1 + S, n);
-    for (int i1 = s1; i1 < s2; i1 += block) {
+    if (fused) {
+      a.ext_minmax = nullptr;
+      const int gend = std::min(s1 + G, n);
+      if (s1 % G == 0 && s1 + block < gend) {  // one group per row: its columns past the first block
+        launch(group_minmax_kernel, static_cast<unsigned>(ceil_div(rows * 32, 256)), 256, 0, st, Wk, rows, n,
+               s1 + block, gend, ext_minmax);
+        a.ext_minmax = ext_minmax;
+      }
+      launch(gptq_superblock_kernel<kBlockLanes>, static_cast<unsigned>(ceil_div(rows, static_cast<int64_t>(rows_cta))),
+             rows_cta * kBlockLanes, super_smem, st, a, s1, s2, block);
+    }
+    for (int i1 = s1; !fused && i1 < s2; i1 += block) {
       a.i1 = i1;
       a.bw = std::min(block, s2 - i1);
       a.e_off = i1 - s1;
