@@ -1108,8 +1108,9 @@ def run_reference(args, world, rank):
 def profile_pass():
     """Two passes of the benchmark layer with an eighth of its tokens (the
     factorization, column loop and packing see the full shapes; X is 268 MB,
-    larger than L2), then the packed-weight matvec 8 times: the command that
-    the ncu summaries under profiles/ capture, one kernel at a time."""
+    larger than L2), then the packed-weight matvec 8 times, then one more
+    pass with the fused row-slab column loop: the command that the ncu
+    summaries under profiles/ capture, one kernel at a time."""
     import torch
 
     import post_weight_quantization_accum_b200 as gq
@@ -1123,6 +1124,11 @@ def profile_pass():
     x = torch.randn(spec.n, device="cuda").to(torch.bfloat16)
     for _ in range(8):
         gq.gptq_dequant_matvec(out["packed"], out["scales"], out["zeros"], spec.n, spec.bits, spec.group, x)
+    gq.gptq_set_column_loop(1)
+    try:
+        gq.quantize_layer(W, X, bits=spec.bits, group=spec.group, damp=spec.damp, block=spec.block)
+    finally:
+        gq.gptq_set_column_loop(0)
     torch.cuda.synchronize()
     print(json.dumps({"profile_pass": "ok", "kernel_launches": gq.gptq_kernel_launches()}))
 
