@@ -342,7 +342,12 @@ size_t gptq_matvec_workspace_size(int32_t n, int32_t batch, gptq_dtype xdt);
  *   y        fp32 [batch, rows], written
  *   ws       gptq_matvec_workspace_size(n, batch, xdt) bytes (256-byte aligned;
  *            may be NULL when that is 0, as it is in this version)
- * Accumulates in fp32.  Asynchronous on `stream`.
+ * Accumulates in fp32.  4-bit codes with bf16 x, n a multiple of 128, groups
+ * of a multiple of 128 columns (or one group per row), no g_idx, and packed
+ * and x 16-byte aligned run on the tensor cores (mma.sync, bf16 operands
+ * 128 + code and x, which are exact; fp32 sums of s (128 + code) x per
+ * 128-column block, the 128 offsets subtracted once per output); every other
+ * case runs the general kernel.  Asynchronous on `stream`.
  * Errors: GPTQ_ERR_INVALID_ARG (sizes, bits not in {2,3,4,8}, group > n,
  * batch outside 1..8, NULL or misaligned pointers, small workspace), before any
  * launch; GPTQ_ERR_CUDA. */
