@@ -575,7 +575,8 @@ gptq_status quantize_layer(const void* W, gptq_dtype wdt, int64_t rows, int n, c
   const int64_t slab = 2 * ceil_div(rows, 2 * static_cast<int64_t>(info->sm_count));
   const bool fused = column_loop_mode() == 1 && S > block && block == kBMax && (block % G == 0 || G == n) &&
                      slab <= kSlabMaxRows;
-  constexpr size_t super_smem = (2 * static_cast<size_t>(kBMax) * BlockShape<kBlockLanes>::kRowPitch + kBMax) * sizeof(float);
+  constexpr size_t super_smem =
+      (2 * static_cast<size_t>(kBMax) * BlockShape<kBlockLanes>::kRowPitch + kBMax) * sizeof(float);
   const int rows_cta = static_cast<int>(std::max<int64_t>(2, slab));
   if (fused) {
     static std::atomic<bool> super_attr[64] = {};
