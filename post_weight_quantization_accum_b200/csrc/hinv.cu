@@ -83,15 +83,24 @@ __global__ void identity_perm_kernel(int32_t* perm, int n) {
 // A's lower triangle at the padded order np: the damped, permuted and
 // reversed Hessian where a, b < n, the identity in the padding.  Dead
 // diagonals become 1 + lambda.  (The upper triangle is never read.)
+constexpr int kGatherRows = 32;  // rows of A per CTA of gather_reversed_kernel
+
+// One thread per column b of A, over a chunk of kGatherRows rows: its source
+// column perm[n-1-b] is read once and the rows' loads are independent of one
+// another, so many are in flight at once.
 __global__ void gather_reversed_kernel(const float* __restrict__ H, const int32_t* __restrict__ perm,
                                        const uint8_t* __restrict__ dead, const double* __restrict__ lambda, int n,
                                        int64_t np, float* __restrict__ A) {
-  for (int64_t a = blockIdx.y; a < np; a += gridDim.y) {
-    const int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (b > a) continue;
+  const int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (b >= np) return;
+  const int pl = b < n ? perm[n - 1 - b] : 0;
+  const int64_t a0 = static_cast<int64_t>(blockIdx.y) * kGatherRows;
+  const int64_t a1 = a0 + kGatherRows < np ? a0 + kGatherRows : np;
+#pragma unroll 8
+  for (int64_t a = a0 > b ? a0 : b; a < a1; ++a) {  // the lower triangle: b <= a
     float v;
     if (a < n && b < n) {
-      const int ph = perm[n - 1 - a], pl = perm[n - 1 - b];
+      const int ph = perm[n - 1 - a];
       if (a == b) {
         const double base = dead[ph] ? 1.0 : static_cast<double>(H[static_cast<size_t>(ph) * n + ph]);
         v = static_cast<float>(base + *lambda);
@@ -935,8 +944,9 @@ gptq_status prepare_hinv(const float* H, const double* hdiag, int n, float damp,
     launch(identity_perm_kernel, static_cast<unsigned>(ceil_div(n, 256)), 256, 0, st, perm, n);
   if (dead_out != nullptr && cudaMemcpyAsync(dead_out, dead, n, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
     return GPTQ_ERR_CUDA;
-  launch(gather_reversed_kernel, dim3(static_cast<unsigned>(ceil_div(np, 256)), static_cast<unsigned>(std::min<int64_t>(np, 65535))),
-         256, 0, st, H, perm, dead, lambda, n, np, A);
+  launch(gather_reversed_kernel,
+         dim3(static_cast<unsigned>(ceil_div(np, 256)), static_cast<unsigned>(ceil_div(np, kGatherRows))), 256, 0, st, H,
+         perm, dead, lambda, n, np, A);
   if (cudaMemsetAsync(Y, 0, static_cast<size_t>(np) * static_cast<size_t>(np) * sizeof(float), st) != cudaSuccess)
     return GPTQ_ERR_CUDA;
   if (launch_status() != GPTQ_OK) return GPTQ_ERR_CUDA;

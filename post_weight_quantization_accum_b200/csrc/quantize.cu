@@ -50,19 +50,24 @@ __device__ __forceinline__ float load_w<float>(const float* p) { return *p; }
 template <>
 __device__ __forceinline__ float load_w<__nv_bfloat16>(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 
-// Wk[r, p] = dead[perm[p]] ? 0 : W[r, perm[p]]  (processing order, fp32);
-// rows along blockIdx.y, so no division per element.
+// Wk[r, p] = dead[perm[p]] ? 0 : W[r, perm[p]]  (processing order, fp32).
+// One thread per column p over a chunk of kGatherRows rows: the column's
+// source index and dead flag are read once, and the rows' loads are
+// independent of one another, so many are in flight at once.
+constexpr int kGatherRows = 16;
+
 template <typename T>
 __global__ void gather_weights_kernel(const T* __restrict__ W, const int32_t* __restrict__ perm,
                                       const uint8_t* __restrict__ dead, int64_t rows, int n, float* __restrict__ Wk) {
-  for (int64_t r = blockIdx.y; r < rows; r += gridDim.y) {
-    const T* src = W + r * n;
-    float* dst = Wk + r * n;
-    for (int p = blockIdx.x * blockDim.x + threadIdx.x; p < n; p += gridDim.x * blockDim.x) {
-      const int c = perm != nullptr ? perm[p] : p;
-      const bool d = dead != nullptr && dead[c];
-      dst[p] = d ? 0.0f : load_w<T>(src + c);
-    }
+  const int p = blockIdx.x * blockDim.x + threadIdx.x;
+  if (p >= n) return;
+  const int c = perm != nullptr ? perm[p] : p;
+  const bool d = dead != nullptr && dead[c];
+  for (int64_t r0 = static_cast<int64_t>(blockIdx.y) * kGatherRows; r0 < rows;
+       r0 += static_cast<int64_t>(gridDim.y) * kGatherRows) {
+    const int64_t r1 = r0 + kGatherRows < rows ? r0 + kGatherRows : rows;
+#pragma unroll 8
+    for (int64_t r = r0; r < r1; ++r) Wk[r * n + p] = d ? 0.0f : load_w<T>(W + r * n + c);
   }
 }
 
@@ -525,8 +530,8 @@ gptq_status quantize_layer(const void* W, gptq_dtype wdt, int64_t rows, int n, c
   const int G = group > 0 ? group : n;
   const int n_groups = static_cast<int>(ceil_div(n, G));
 
-  const dim3 gg(static_cast<unsigned>(std::min<int64_t>(ceil_div(n, 256), 64)),
-                static_cast<unsigned>(std::min<int64_t>(rows, 65535)));
+  const dim3 gg(static_cast<unsigned>(ceil_div(n, 256)),
+                static_cast<unsigned>(std::min<int64_t>(ceil_div(rows, static_cast<int64_t>(kGatherRows)), 65535)));
   if (wdt == GPTQ_BF16)
     launch(gather_weights_kernel<__nv_bfloat16>, gg, 256, 0, st, static_cast<const __nv_bfloat16*>(W), perm, dead, rows,
                                                              n, Wk);
