@@ -49,6 +49,22 @@ def test_pure_calls(lib):
     assert lib.gptq_version() == 100
 
 
+def test_column_loop_selector(lib):
+    """gptq_set_column_loop: 0 (per-block loop) by default, 1 selects the fused
+    row-slab pass, anything else falls back to 0; the setting needs no GPU."""
+    lib.gptq_get_column_loop.restype = ctypes.c_int32
+    lib.gptq_set_column_loop.argtypes = [ctypes.c_int32]
+    assert lib.gptq_get_column_loop() == 0
+    try:
+        lib.gptq_set_column_loop(1)
+        assert lib.gptq_get_column_loop() == 1
+        for other in (2, -1, 7):
+            lib.gptq_set_column_loop(other)
+            assert lib.gptq_get_column_loop() == 0
+    finally:
+        lib.gptq_set_column_loop(0)
+
+
 def test_invalid_arguments_rejected_before_any_launch(lib):
     P = ctypes.c_void_p
     f = lib.gptq_quantize_layer
